@@ -1,0 +1,235 @@
+"""Seeded synthetic inputs for the FFD decode path.
+
+This module only draws random numbers and lays them out; it holds none of the
+method's arithmetic (no quantisation, no scoring, no selection, no softmax).
+Both the CPU oracle and the CUDA path consume the arrays it returns, so the two
+sides always see bit-identical inputs.
+
+Workloads follow the five synthetic decode shapes used throughout the project
+(tiny / Llama-3-8B-shaped / 128K long context with drift / 256K max context /
+ragged serving batch).  The pages measure on RULER and LongBench (Faster Than
+Flash, gist.science explainer, "Key Results"); those suites are not available
+here, and these planted-needle and drift inputs stand in for their needle and
+long-context structure.
+
+Recipe (all float work in fp32, one final round-to-nearest-even to bf16):
+  * q, K, V ~ N(0, 1), drawn with numpy's PCG64 generator seeded through
+    SeedSequence(seed, spawn_key=(stream, batch, kv-head)); every (tensor, batch,
+    kv-head) row has its own independent stream, so rows can be drawn in any
+    order or in parallel.
+  * drift (long-context workload only): per (kv-head, channel) a random walk
+    D_t = D_{t-1} + sigma * xi_t, D_{-1} = 0, added to the keys.
+  * needles: distinct full-block indices drawn without replacement; planted in
+    every kv-head; needle i in kv-head g targets query head g*G + (i mod G); every
+    key row of the block gets + 3 * q_h / |q_h|.
+  * tokens at or beyond each sequence's length (the unused cache tail) hold
+    finite poison values, so that a kernel that reads past the length fails.
+"""
+from __future__ import annotations
+
+import concurrent.futures
+import dataclasses
+import os
+from typing import Dict, List, Optional
+
+import numpy as np
+
+HEAD_DIM = 128
+
+# Finite poison written into the cache tail (positions >= length).
+TAIL_K_VALUE = 8.0
+TAIL_V_VALUE = 1000.0
+# Poison for packed-key bytes and scale entries that no quantise call writes.
+PACKED_POISON_BYTE = 0xFF
+SCALE_POISON_BF16 = 0x4000  # 2.0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    capacity: int  # tokens per (batch, kv-head) row of the cache
+    block_size: int
+    split_blocks: int
+    delta: float
+    seed: int
+    context: Optional[int] = None  # fixed length for every sequence
+    ragged: Optional[tuple] = None  # (lo, hi) inclusive uniform lengths
+    needles: Optional[int] = None  # needle blocks per sequence
+    needle_every: Optional[int] = None  # needles = length // needle_every
+    drift_sigma: float = 0.0
+    head_dim: int = HEAD_DIM
+    description: str = ""
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    def shape_dict(self) -> dict:
+        return dict(batch=self.batch, num_q_heads=self.num_q_heads,
+                    num_kv_heads=self.num_kv_heads, head_dim=self.head_dim,
+                    capacity=self.capacity, block_size=self.block_size,
+                    split_blocks=self.split_blocks)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": Workload(
+        name="tiny", batch=1, num_q_heads=4, num_kv_heads=1, capacity=4096,
+        block_size=64, split_blocks=16, delta=2.0, seed=0, context=4096,
+        needles=2,
+        description="B1 Hq4 Hkv1 D128 N4096 T64 S16 delta2, 2 needles"),
+    "llama": Workload(
+        name="llama", batch=4, num_q_heads=32, num_kv_heads=8, capacity=32768,
+        block_size=64, split_blocks=32, delta=3.0, seed=1, context=32768,
+        needles=8,
+        description="Llama-3-8B-shaped: B4 Hq32 Hkv8 D128 N32768 T64 S32 delta3, 8 needles/seq"),
+    "long128k": Workload(
+        name="long128k", batch=1, num_q_heads=32, num_kv_heads=8, capacity=131072,
+        block_size=64, split_blocks=64, delta=3.0, seed=2, context=131072,
+        needles=16, drift_sigma=0.05,
+        description="long context: B1 Hq32 Hkv8 D128 N131072 T64 S64 delta3, drift 0.05/token, 16 needles"),
+    "max256k": Workload(
+        name="max256k", batch=1, num_q_heads=32, num_kv_heads=8, capacity=262144,
+        block_size=128, split_blocks=64, delta=3.0, seed=3, context=262144,
+        needles=32,
+        description="max context: B1 Hq32 Hkv8 D128 N262144 T128 S64, delta sweep {1,2,3,4,inf}, 32 needles"),
+    "ragged": Workload(
+        name="ragged", batch=16, num_q_heads=32, num_kv_heads=8, capacity=65536,
+        block_size=64, split_blocks=32, delta=3.0, seed=4, ragged=(8192, 65536),
+        needle_every=4096,
+        description="ragged serving batch: B16 Hq32 Hkv8 D128 len~U[8192,65536] T64 S32 delta3, needles=len/4096"),
+}
+
+MAX256K_DELTAS = (1.0, 2.0, 3.0, 4.0, float("inf"))
+
+_STREAM_Q, _STREAM_K, _STREAM_V, _STREAM_DRIFT, _STREAM_META = 1, 2, 3, 4, 5
+
+
+def _rng(seed: int, stream: int, b: int = 0, g: int = 0) -> np.random.Generator:
+    ss = np.random.SeedSequence(entropy=seed, spawn_key=(stream, b, g))
+    return np.random.Generator(np.random.PCG64(ss))
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (nearest, ties to even); finite inputs only."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = ((u >> 16) & 1) + np.uint32(0x7FFF)
+    return ((u + rounding) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(h: np.ndarray) -> np.ndarray:
+    return (np.asarray(h, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _bf16_scalar_bits(v: float) -> int:
+    return int(f32_to_bf16_bits(np.array([v], dtype=np.float32))[0])
+
+
+def draw_lengths(w: Workload) -> np.ndarray:
+    if w.ragged is not None:
+        lo, hi = w.ragged
+        return _rng(w.seed, _STREAM_META).integers(lo, hi, endpoint=True,
+                                                   size=w.batch).astype(np.int32)
+    ctx = w.capacity if w.context is None else w.context
+    return np.full(w.batch, ctx, dtype=np.int32)
+
+
+def draw_needles(w: Workload, lengths: np.ndarray) -> List[np.ndarray]:
+    """Sorted needle block indices per sequence (full blocks only)."""
+    out = []
+    for b in range(w.batch):
+        n_full = int(lengths[b]) // w.block_size
+        if w.needle_every is not None:
+            count = int(lengths[b]) // w.needle_every
+        else:
+            count = w.needles or 0
+        count = min(count, n_full)
+        rng = _rng(w.seed, _STREAM_META, b + 1, 0)
+        out.append(np.sort(rng.choice(n_full, size=count, replace=False)).astype(np.int64)
+                   if count > 0 else np.zeros(0, dtype=np.int64))
+    return out
+
+
+def make_inputs(w: Workload, lengths: Optional[np.ndarray] = None,
+                with_needles: bool = True) -> dict:
+    """Draw one decode step's inputs for workload ``w``.
+
+    Returns a dict of numpy arrays: ``q`` [B,Hq,D], ``k`` and ``v`` [B,Hkv,cap,D]
+    (bf16 bit patterns as uint16), ``lengths`` int32 [B] and ``needles`` (list of
+    block-index arrays per sequence).
+    """
+    B, Hq, Hkv, cap, D = w.batch, w.num_q_heads, w.num_kv_heads, w.capacity, w.head_dim
+    G = Hq // Hkv
+    if lengths is None:
+        lengths = draw_lengths(w)
+    lengths = np.asarray(lengths, dtype=np.int32)
+    needles = draw_needles(w, lengths) if with_needles else [np.zeros(0, np.int64)] * B
+
+    q32 = np.empty((B, Hq, D), dtype=np.float32)
+    for b in range(B):
+        q32[b] = _rng(w.seed, _STREAM_Q, b).standard_normal((Hq, D), dtype=np.float32)
+    q = f32_to_bf16_bits(q32)
+    qf = bf16_bits_to_f32(q)  # the query the path actually sees
+
+    k = np.empty((B, Hkv, cap, D), dtype=np.uint16)
+    v = np.empty((B, Hkv, cap, D), dtype=np.uint16)
+    tail_k = _bf16_scalar_bits(TAIL_K_VALUE)
+    tail_v = _bf16_scalar_bits(TAIL_V_VALUE)
+
+    def fill_row(bg):
+        b, g = bg
+        n = int(lengths[b])
+        kk = _rng(w.seed, _STREAM_K, b, g).standard_normal((n, D), dtype=np.float32)
+        if w.drift_sigma > 0.0 and n > 0:
+            # random walk per channel, accumulated along the token axis
+            steps = _rng(w.seed, _STREAM_DRIFT, b, g).standard_normal((D, n), dtype=np.float32)
+            steps *= np.float32(w.drift_sigma)
+            kk += np.cumsum(steps, axis=1, dtype=np.float32).T
+        for i, j in enumerate(needles[b]):
+            h = g * G + (i % G)
+            qh = qf[b, h]
+            norm = np.float32(np.sqrt(np.sum(qh * qh, dtype=np.float32)))
+            direction = (np.float32(3.0) * qh / norm).astype(np.float32)
+            t0 = int(j) * w.block_size
+            kk[t0:t0 + w.block_size] += direction
+        k[b, g, :n] = f32_to_bf16_bits(kk)
+        k[b, g, n:] = tail_k
+        vv = _rng(w.seed, _STREAM_V, b, g).standard_normal((n, D), dtype=np.float32)
+        v[b, g, :n] = f32_to_bf16_bits(vv)
+        v[b, g, n:] = tail_v
+
+    rows = [(b, g) for b in range(B) for g in range(Hkv)]
+    workers = max(1, min(len(rows), os.cpu_count() or 1, 16))
+    if workers == 1:
+        for bg in rows:
+            fill_row(bg)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(fill_row, rows))
+    return dict(q=q, k=k, v=v, lengths=lengths, needles=needles)
+
+
+def scaled_workload(w: Workload, **overrides) -> Workload:
+    """Copy of ``w`` with some fields replaced (used for small parity cases)."""
+    return dataclasses.replace(w, **overrides)
+
+
+def random_small_workload(seed: int, batch: int, group: int, num_kv_heads: int,
+                          capacity: int, block_size: int, split_blocks: int,
+                          delta: float, lengths_lo: int, lengths_hi: int,
+                          needles: int = 1) -> Workload:
+    """A small randomly-shaped workload for sweeps (ragged lengths, any split)."""
+    return Workload(name=f"rand{seed}", batch=batch, num_q_heads=group * num_kv_heads,
+                    num_kv_heads=num_kv_heads, capacity=capacity, block_size=block_size,
+                    split_blocks=split_blocks, delta=delta, seed=1000 + seed,
+                    ragged=(lengths_lo, lengths_hi), needles=needles)
+
+
+def poison_packed(shape_packed) -> np.ndarray:
+    return np.full(shape_packed, PACKED_POISON_BYTE, dtype=np.uint8)
+
+
+def poison_scales(shape_scales) -> np.ndarray:
+    return np.full(shape_scales, SCALE_POISON_BF16, dtype=np.uint16)
