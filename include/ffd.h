@@ -1,0 +1,161 @@
+/*
+ * ffd.h -- C ABI of the B200 (sm_100a) Faster Flash Decoding decode path.
+ *
+ * Method: "Faster Than Flash: Exploiting Attention Sparsity for Efficient
+ * Long-Context Decoding" (arXiv 2609.00097).  Single-token decode attention
+ * over a long KV cache with a fused selector and computer: the selector scans
+ * a low-bit copy of the keys (gist.science explainer, Methodology 1
+ * "Content-Aware Scanning via Low-Bit Quantization"), keeps the blocks whose
+ * tentative score lies within delta of a reference maximum (Methodology 2
+ * "The Top-delta Selection Strategy"), and the computer runs exact attention
+ * over the kept blocks only (Methodology 3, stage "Fine-Grained Refinement");
+ * both live in one kernel (arXiv abstract: selector and computer "in a fully
+ * fused kernel", scan results reused for computation).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are caller-owned device memory unless stated otherwise; the
+ *     library allocates nothing and keeps no state between calls.
+ *   - Every device pointer must be 16-byte aligned; tensors are dense,
+ *     row-major, in the layouts given below.
+ *   - bf16 means IEEE bfloat16 bit patterns (uint16).
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and may be captured into a CUDA graph.  Per-sequence
+ *     lengths live on the device, so no call reads device memory from the host.
+ *   - Host-side argument checks fail before any launch and return a status;
+ *     no entry point throws or aborts.  Length values are checked on the
+ *     device (see ffd_decode).
+ *
+ * Shapes (symbols): B batch, Hq query heads, Hkv kv heads, G = Hq / Hkv,
+ * D = 128 head dim, T block tokens, S split blocks, cap tokens per cache row,
+ * nblk = cap / T, W = ceil(nblk / 32) mask words per (b, kv-head).
+ *
+ * Data layouts
+ *   q        bf16 [B][Hq][D]                  query head h uses kv-head h / G
+ *   k, v     bf16 [B][Hkv][cap][D]            the KV cache
+ *   k_packed u8   [B][Hkv][cap][D/2]          int4 key copy: byte i of a token
+ *            row holds channel 2i in the low nibble and channel 2i+1 in the high
+ *            nibble, each as code + 8 with code in [-7, 7]
+ *   k_scales bf16 [B][Hkv][nblk][D]           per-block-per-channel key scales
+ *   lengths  int32 [B] (device)               valid tokens per sequence
+ *   out      bf16 [B][Hq][D]
+ *   mask     u32  [B][Hkv][W]                 bit (j % 32) of word j / 32 set iff
+ *            block j was selected for that kv-head; bits >= ceil(len/T) are 0
+ */
+#ifndef FFD_H
+#define FFD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FFD_OK = 0,
+  FFD_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape, NaN or negative delta */
+  FFD_ERR_UNSUPPORTED = 2,  /* a valid shape this build does not implement */
+  FFD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than ffd_decode_workspace_bytes */
+  FFD_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, tensor map) */
+  FFD_ERR_DEVICE_CHECK = 5, /* ffd_check_device_status found a device-side error flag */
+  FFD_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up */
+} ffd_status;
+
+/* Device-side error flags, reported by ffd_check_device_status. */
+#define FFD_DEVICE_FLAG_BAD_LENGTH 0x1u /* some lengths[b] outside [0, cap] */
+#define FFD_DEVICE_FLAG_TIMEOUT 0x2u    /* a bounded barrier wait expired */
+
+/* block_begin value for ffd_quantize_keys: each sequence's last block only. */
+#define FFD_LAST_BLOCK (-1)
+
+/* Largest split size (blocks) this build accepts. */
+#define FFD_MAX_SPLIT_BLOCKS 512
+
+typedef struct {
+  int32_t batch;        /* B >= 0 */
+  int32_t num_q_heads;  /* Hq > 0, multiple of num_kv_heads */
+  int32_t num_kv_heads; /* Hkv in [1, 65535] */
+  int32_t head_dim;     /* D, must be 128 */
+  int32_t capacity;     /* cap >= 0, multiple of block_size */
+  int32_t block_size;   /* T: 64 or 128 */
+  int32_t split_blocks; /* S in [1, FFD_MAX_SPLIT_BLOCKS] */
+} ffd_shape;
+
+/* Bytes of k_packed, k_scales; words of mask (all for the whole batch).
+ * Return 0 for an invalid shape. */
+size_t ffd_packed_bytes(const ffd_shape *shape);
+size_t ffd_scale_bytes(const ffd_shape *shape);
+size_t ffd_mask_words(const ffd_shape *shape);
+
+/* Device workspace ffd_decode needs: split partials (running max, sum and
+ * unnormalised output per head), per-split selection bits, one arrival
+ * counter per (b, kv-head) and the sticky device error word.  0 for an
+ * invalid shape. */
+size_t ffd_decode_workspace_bytes(const ffd_shape *shape);
+
+/* Zero a workspace (cudaMemsetAsync on the stream).  Call once after
+ * allocating it; ffd_decode leaves it ready for the next call. */
+ffd_status ffd_workspace_init(const ffd_shape *shape, void *workspace,
+                              size_t workspace_bytes, void *cuda_stream);
+
+/* Low-bit key copy (gist.science explainer, Methodology 1: keys are kept as a
+ * low-bit "thumbnail" used only for scanning; here int4 with per-block-per-
+ * channel bf16 scales).  For every (b, kv-head) and every block j with
+ * block_begin <= j < ceil(lengths[b] / T) -- or only j = ceil(lengths[b]/T) - 1
+ * when block_begin == FFD_LAST_BLOCK -- over the block's valid tokens t:
+ *   amax_c  = max_t |k[t][c]|,  s_c = bf16_rne(amax_c / 7)   (IEEE fp32 division)
+ *   code    = s_c == 0 ? 0 : clamp(rint_even(k[t][c] / s_c), -7, 7)
+ * Tokens at or beyond lengths[b] in the last block get code 0 and do not
+ * enter amax.  Blocks outside that range are not written.  Sequences whose
+ * length is outside [0, cap] are skipped (ffd_decode reports them).
+ * Run it once over the whole cache after prefill (block_begin = 0) and with
+ * FFD_LAST_BLOCK after each appended token. */
+ffd_status ffd_quantize_keys(const ffd_shape *shape, const void *k_bf16,
+                             const int32_t *d_lengths, int32_t block_begin,
+                             void *k_packed, void *k_scales, void *cuda_stream);
+
+/* One fused decode step (selector + computer + split merge, one launch).
+ *
+ * Selector (skipped when delta == +INFINITY):
+ *   per (b, query head h, block j): p_c = q_c * s_{j,c} (fp32),
+ *   a = max_c |p_c|, qi_c = clamp(rint_even(p_c * (127 / a)), -127, 127) (int8),
+ *   cf = (a / 127) * (1 / sqrt(128)); I_t = sum_c qi_c * code_{t,c} (exact int),
+ *   score_j = float(max over valid t of I_t) * cf   (a == 0 gives score 0).
+ *   Blocks are cut into splits of S consecutive blocks (split s holds blocks
+ *   [sS, min((s+1)S, nb))); inside a split, in ascending order,
+ *   m = max(m, score_j) and block j is kept for head h iff score_j >= m - delta
+ *   (Methodology 2, Mechanism, with the running maximum of the split as the
+ *   reference: no synchronisation across splits).  A kv-head keeps the union
+ *   over its G query heads; delta is in natural-log logit units (after
+ *   1/sqrt(D)), delta = 0 keeps running-maximum records only, and the first
+ *   block of every split is always kept.
+ * Computer: every query head of the group attends (softmax(q.K/sqrt(D)) V,
+ *   fp32 accumulation, bf16 output) over the valid tokens of the kept blocks;
+ *   splits are merged with log-sum-exp.  delta == +INFINITY is dense
+ *   flash-decoding over all valid tokens (k_packed, k_scales may be NULL).
+ *
+ * A sequence with lengths[b] == 0 yields zero output rows and an empty mask.
+ * lengths[b] outside [0, cap] sets FFD_DEVICE_FLAG_BAD_LENGTH in the
+ * workspace and yields zero rows and an empty mask for that sequence.
+ * Steps that share a workspace must not overlap on the GPU. */
+ffd_status ffd_decode(const ffd_shape *shape, const void *q_bf16, const void *k_bf16,
+                      const void *v_bf16, const void *k_packed, const void *k_scales,
+                      const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                      void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+/* Synchronise the stream, read and clear the workspace's sticky device error
+ * word.  *flags_out (may be NULL) receives FFD_DEVICE_FLAG_* bits.  Returns
+ * FFD_ERR_DEVICE_CHECK if any flag was set, FFD_ERR_CUDA on a CUDA error. */
+ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream);
+
+/* Static description of a status code. */
+const char *ffd_status_string(ffd_status status);
+
+/* ABI version of this library (bumped on any incompatible change). */
+int32_t ffd_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FFD_H */

@@ -1,0 +1,254 @@
+// api.cu -- the C ABI declared in include/ffd.h: host-side validation,
+// workspace layout, TMA descriptors and kernel launches.  No entry point
+// allocates memory or synchronises, except ffd_check_device_status.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ffd.h"
+#include "ffd_internal.h"
+
+namespace ffd {
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ffd_status check_shape(const ffd_shape *s) {
+  if (s == nullptr) return FFD_ERR_INVALID_ARG;
+  if (s->batch < 0 || s->num_q_heads <= 0 || s->num_kv_heads <= 0 || s->capacity < 0 ||
+      s->head_dim <= 0 || s->block_size <= 0 || s->split_blocks <= 0)
+    return FFD_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads != 0) return FFD_ERR_INVALID_ARG;
+  if (s->capacity % s->block_size != 0) return FFD_ERR_INVALID_ARG;
+  if (s->head_dim != kHeadDim) return FFD_ERR_UNSUPPORTED;
+  if (s->block_size != 64 && s->block_size != 128) return FFD_ERR_UNSUPPORTED;
+  if (s->split_blocks > FFD_MAX_SPLIT_BLOCKS) return FFD_ERR_UNSUPPORTED;
+  const int g = s->num_q_heads / s->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return FFD_ERR_UNSUPPORTED;
+  if (s->num_kv_heads > 65535 || s->batch > 65535) return FFD_ERR_UNSUPPORTED;
+  // token rows are addressed with 32-bit TMA coordinates
+  if (static_cast<int64_t>(s->batch) * s->num_kv_heads * s->capacity >= (int64_t{1} << 31))
+    return FFD_ERR_UNSUPPORTED;
+  return FFD_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// K or V cache viewed as rows of 128 bf16 (256 bytes); 64 x 64 boxes with
+// the 128-byte swizzle (one box = one 64-channel half of a 64-token tile).
+bool make_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), rows > 0 ? rows : 1};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                            strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group, int32_t capacity,
+                                 int32_t block_size, int32_t split_blocks) {
+  WorkspaceLayout L{};
+  const int64_t nblk = capacity / block_size;
+  L.nsplit_max = static_cast<int32_t>((nblk + split_blocks - 1) / split_blocks);
+  L.split_words = (split_blocks + 31) / 32;
+  const size_t rows = static_cast<size_t>(batch) * num_kv_heads;
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.counters = off;
+  off += round_up(rows * 4, 256);
+  L.split_bits = off;
+  off += round_up(rows * L.nsplit_max * L.split_words * 4, 256);
+  L.partials = off;
+  off += rows * L.nsplit_max * group * kPartialStride * 4;
+  L.total = round_up(off, 256);
+  return L;
+}
+
+}  // namespace ffd
+
+using namespace ffd;
+
+extern "C" {
+
+int32_t ffd_abi_version(void) { return kAbiVersion; }
+
+const char *ffd_status_string(ffd_status status) {
+  switch (status) {
+    case FFD_OK: return "ok";
+    case FFD_ERR_INVALID_ARG: return "invalid argument";
+    case FFD_ERR_UNSUPPORTED: return "unsupported shape";
+    case FFD_ERR_WORKSPACE: return "workspace missing or too small";
+    case FFD_ERR_CUDA: return "CUDA runtime error";
+    case FFD_ERR_DEVICE_CHECK: return "device-side error flag set";
+    case FFD_ERR_TIMEOUT: return "bounded device wait expired";
+  }
+  return "unknown status";
+}
+
+size_t ffd_packed_bytes(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->num_kv_heads * s->capacity * (kHeadDim / 2);
+}
+
+size_t ffd_scale_bytes(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->num_kv_heads * (s->capacity / s->block_size) * kHeadDim * 2;
+}
+
+size_t ffd_mask_words(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  const size_t nblk = s->capacity / s->block_size;
+  return static_cast<size_t>(s->batch) * s->num_kv_heads * ((nblk + 31) / 32);
+}
+
+size_t ffd_decode_workspace_bytes(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  return workspace_layout(s->batch, s->num_kv_heads, s->num_q_heads / s->num_kv_heads, s->capacity,
+                          s->block_size, s->split_blocks)
+      .total;
+}
+
+ffd_status ffd_workspace_init(const ffd_shape *s, void *workspace, size_t workspace_bytes,
+                              void *cuda_stream) {
+  ffd_status st = check_shape(s);
+  if (st != FFD_OK) return st;
+  const size_t need = ffd_decode_workspace_bytes(s);
+  if (workspace == nullptr || workspace_bytes < need) return FFD_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FFD_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, need, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return FFD_ERR_CUDA;
+  return FFD_OK;
+}
+
+ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32_t *d_lengths,
+                             int32_t block_begin, void *k_packed, void *k_scales, void *cuda_stream) {
+  ffd_status st = check_shape(s);
+  if (st != FFD_OK) return st;
+  if (block_begin < FFD_LAST_BLOCK) return FFD_ERR_INVALID_ARG;
+  const int nblk = s->capacity / s->block_size;
+  if (s->batch == 0 || nblk == 0) return FFD_OK;
+  if (k_bf16 == nullptr || d_lengths == nullptr || k_packed == nullptr || k_scales == nullptr)
+    return FFD_ERR_INVALID_ARG;
+  if (!aligned16(k_bf16) || !aligned16(k_packed) || !aligned16(k_scales) ||
+      (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
+    return FFD_ERR_INVALID_ARG;
+  const int blocks = block_begin < 0 ? 1 : nblk - block_begin;
+  if (blocks <= 0) return FFD_OK;
+  QuantizeParams p{};
+  p.k = static_cast<const uint16_t *>(k_bf16);
+  p.lengths = d_lengths;
+  p.packed = static_cast<uint8_t *>(k_packed);
+  p.scales = static_cast<uint16_t *>(k_scales);
+  p.batch = s->batch;
+  p.num_kv_heads = s->num_kv_heads;
+  p.capacity = s->capacity;
+  p.block_begin = block_begin;
+  const dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(s->num_kv_heads),
+                  static_cast<unsigned>(s->batch));
+  if (launch_quantize(p, s->block_size, grid, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return FFD_ERR_CUDA;
+  return FFD_OK;
+}
+
+ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                      const void *k_packed, const void *k_scales, const int32_t *d_lengths, float delta,
+                      void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
+                      void *cuda_stream) {
+  ffd_status st = check_shape(s);
+  if (st != FFD_OK) return st;
+  if (std::isnan(delta) || delta < 0.0f) return FFD_ERR_INVALID_ARG;
+  if (s->batch == 0) return FFD_OK;
+  const bool dense = std::isinf(delta);
+  const int group = s->num_q_heads / s->num_kv_heads;
+  const WorkspaceLayout L =
+      workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks);
+  if (workspace == nullptr || workspace_bytes < L.total) return FFD_ERR_WORKSPACE;
+  if (q_bf16 == nullptr || k_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
+      out_bf16 == nullptr || mask == nullptr)
+    return FFD_ERR_INVALID_ARG;
+  if (!dense && (k_packed == nullptr || k_scales == nullptr)) return FFD_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
+      !aligned16(mask) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
+    return FFD_ERR_INVALID_ARG;
+  if (!dense && (!aligned16(k_packed) || !aligned16(k_scales))) return FFD_ERR_INVALID_ARG;
+
+  const uint64_t rows = static_cast<uint64_t>(s->batch) * s->num_kv_heads * s->capacity;
+  CUtensorMap tmap_k, tmap_v;
+  if (!make_kv_tensor_map(&tmap_k, k_bf16, rows) || !make_kv_tensor_map(&tmap_v, v_bf16, rows))
+    return FFD_ERR_CUDA;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t *>(q_bf16);
+  p.packed = static_cast<const uint8_t *>(k_packed);
+  p.scales = static_cast<const uint16_t *>(k_scales);
+  p.lengths = d_lengths;
+  p.out = static_cast<uint16_t *>(out_bf16);
+  p.mask = mask;
+  p.err = reinterpret_cast<uint32_t *>(ws + L.err);
+  p.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+  p.split_bits = reinterpret_cast<uint32_t *>(ws + L.split_bits);
+  p.partials = reinterpret_cast<float *>(ws + L.partials);
+  p.batch = s->batch;
+  p.num_kv_heads = s->num_kv_heads;
+  p.capacity = s->capacity;
+  p.split_blocks = s->split_blocks;
+  p.nsplit_max = L.nsplit_max;
+  p.mask_words = static_cast<int32_t>((s->capacity / s->block_size + 31) / 32);
+  p.split_words = L.split_words;
+  p.delta = delta;
+  p.dense = dense ? 1 : 0;
+
+  const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
+                  static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
+  const size_t smem = decode_smem_bytes(s->block_size, group, s->split_blocks);
+  if (launch_decode(p, tmap_k, tmap_v, s->block_size, group, grid, smem,
+                    static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return FFD_ERR_CUDA;
+  return FFD_OK;
+}
+
+ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream) {
+  if (workspace == nullptr || !aligned16(workspace)) return FFD_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint32_t flags = 0;
+  if (cudaMemcpyAsync(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return FFD_ERR_CUDA;
+  if (flags != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(flags), stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return FFD_ERR_CUDA;
+  }
+  if (flags_out) *flags_out = flags;
+  return flags != 0 ? FFD_ERR_DEVICE_CHECK : FFD_OK;
+}
+
+}  // extern "C"

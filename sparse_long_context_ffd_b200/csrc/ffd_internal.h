@@ -1,0 +1,71 @@
+// ffd_internal.h -- kernel parameter blocks and launchers shared between the
+// host entry points (api.cu) and the kernels (quantize.cu, decode.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace ffd {
+
+constexpr int kHeadDim = 128;
+constexpr int kPackedRowBytes = kHeadDim / 2;  // 64 bytes of nibbles per token
+constexpr int kScaleRowBytes = kHeadDim * 2;   // 128 bf16 scales per block
+
+// Fused decode kernel geometry.
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kSubTokens = 64;                             // K/V tokens per pipeline stage
+constexpr int kKvStageBytes = 4 * kSubTokens * 64 * 2;     // K lo/hi + V lo/hi halves, 32 KiB
+constexpr int kKvStages = 3;
+constexpr int kRingBytes = kKvStages * kKvStageBytes;  // 96 KiB, reused by the scan
+constexpr int kPartialStride = 132;                    // floats per (split, head): acc[128], m, l
+constexpr uint64_t kWaitLimitNs = 2000000000ull;       // bounded mbarrier waits (2 s)
+
+constexpr uint32_t kFlagBadLength = 0x1u;
+constexpr uint32_t kFlagTimeout = 0x2u;
+
+struct DecodeParams {
+  const uint16_t *q;       // bf16 [B][Hq][D]
+  const uint8_t *packed;   // [B][Hkv][cap][64]
+  const uint16_t *scales;  // bf16 [B][Hkv][nblk][D]
+  const int32_t *lengths;  // [B]
+  uint16_t *out;           // bf16 [B][Hq][D]
+  uint32_t *mask;          // [B][Hkv][mask_words]
+  uint32_t *err;           // sticky device flags
+  uint32_t *counters;      // [B][Hkv]
+  uint32_t *split_bits;    // [B][Hkv][nsplit_max][split_words]
+  float *partials;         // [B][Hkv][nsplit_max][G][kPartialStride]
+  int32_t batch, num_kv_heads, capacity, split_blocks, nsplit_max, mask_words, split_words;
+  float delta;
+  int32_t dense;
+};
+
+struct QuantizeParams {
+  const uint16_t *k;
+  const int32_t *lengths;
+  uint8_t *packed;
+  uint16_t *scales;
+  int32_t batch, num_kv_heads, capacity, block_begin;
+};
+
+// Workspace carve-up (byte offsets), identical on host and device.
+struct WorkspaceLayout {
+  size_t err, counters, split_bits, partials, total;
+  int32_t nsplit_max, split_words;
+};
+
+WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group,
+                                 int32_t capacity, int32_t block_size, int32_t split_blocks);
+
+size_t decode_smem_bytes(int block_size, int group, int split_blocks);
+
+cudaError_t launch_quantize(const QuantizeParams &p, int block_size, dim3 grid,
+                            cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k,
+                          const CUtensorMap &tmap_v, int block_size, int group, dim3 grid,
+                          size_t smem_bytes, cudaStream_t stream);
+
+}  // namespace ffd

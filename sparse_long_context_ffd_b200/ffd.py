@@ -1,0 +1,199 @@
+"""Thin ctypes binding of the C ABI in include/ffd.h (argument marshalling only).
+
+Every step of the decode path runs in the CUDA library; this module only turns
+torch tensors into pointers, picks the current CUDA stream and maps status
+codes to exceptions.  There is no fallback: if the library is missing and
+cannot be built, importing a function raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional
+
+from . import build as _build
+
+FFD_OK = 0
+FFD_ERR_INVALID_ARG = 1
+FFD_ERR_UNSUPPORTED = 2
+FFD_ERR_WORKSPACE = 3
+FFD_ERR_CUDA = 4
+FFD_ERR_DEVICE_CHECK = 5
+FFD_ERR_TIMEOUT = 6
+
+FFD_DEVICE_FLAG_BAD_LENGTH = 0x1
+FFD_DEVICE_FLAG_TIMEOUT = 0x2
+FFD_LAST_BLOCK = -1
+FFD_MAX_SPLIT_BLOCKS = 512
+
+# Every function the header declares; the library must export all of them.
+EXPORTED = (
+    "ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words", "ffd_decode_workspace_bytes",
+    "ffd_workspace_init", "ffd_quantize_keys", "ffd_decode", "ffd_check_device_status",
+    "ffd_status_string", "ffd_abi_version",
+)
+
+
+class FFDError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("capacity", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("split_blocks", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "Shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_shape(batch, num_q_heads, num_kv_heads, capacity, block_size, split_blocks,
+               head_dim=128) -> Shape:
+    return Shape(batch, num_q_heads, num_kv_heads, head_dim, capacity, block_size, split_blocks)
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libffd_b200.so, building it with nvcc first if it is missing or stale."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if _build.is_stale():
+                _build.build()
+            lib = ctypes.CDLL(_build.LIB)
+            sp = ctypes.POINTER(Shape)
+            p, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+            for name in ("ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words",
+                         "ffd_decode_workspace_bytes"):
+                getattr(lib, name).argtypes = [sp]
+                getattr(lib, name).restype = sz
+            lib.ffd_workspace_init.argtypes = [sp, p, sz, p]
+            lib.ffd_workspace_init.restype = st
+            lib.ffd_quantize_keys.argtypes = [sp, p, p, ctypes.c_int32, p, p, p]
+            lib.ffd_quantize_keys.restype = st
+            lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
+            lib.ffd_decode.restype = st
+            lib.ffd_check_device_status.argtypes = [p, ctypes.POINTER(ctypes.c_uint32), p]
+            lib.ffd_check_device_status.restype = st
+            lib.ffd_status_string.argtypes = [st]
+            lib.ffd_status_string.restype = ctypes.c_char_p
+            lib.ffd_abi_version.argtypes = []
+            lib.ffd_abi_version.restype = ctypes.c_int32
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().ffd_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return int(load_library().ffd_abi_version())
+
+
+def _check(status: int, what: str) -> None:
+    if status != FFD_OK:
+        raise FFDError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a CUDA tensor (None passes a null pointer)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("FFD entry points take CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("FFD entry points take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def packed_bytes(shape: Shape) -> int:
+    return int(load_library().ffd_packed_bytes(ctypes.byref(shape)))
+
+
+def scale_bytes(shape: Shape) -> int:
+    return int(load_library().ffd_scale_bytes(ctypes.byref(shape)))
+
+
+def mask_words(shape: Shape) -> int:
+    return int(load_library().ffd_mask_words(ctypes.byref(shape)))
+
+
+def decode_workspace_bytes(shape: Shape) -> int:
+    return int(load_library().ffd_decode_workspace_bytes(ctypes.byref(shape)))
+
+
+def workspace_init(shape: Shape, workspace, stream=None) -> None:
+    _check(load_library().ffd_workspace_init(ctypes.byref(shape), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(),
+                                             _stream(stream)), "ffd_workspace_init")
+
+
+def quantize_keys(shape: Shape, k, lengths, block_begin: int, k_packed, k_scales,
+                  stream=None) -> None:
+    _check(load_library().ffd_quantize_keys(ctypes.byref(shape), _ptr(k), _ptr(lengths),
+                                            int(block_begin), _ptr(k_packed), _ptr(k_scales),
+                                            _stream(stream)), "ffd_quantize_keys")
+
+
+def decode(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out, mask,
+           workspace, stream=None) -> None:
+    _check(load_library().ffd_decode(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
+                                      float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream(stream)), "ffd_decode")
+
+
+def check_device_status(workspace, stream=None) -> int:
+    """Synchronise, read and clear the device flags; returns FFD_DEVICE_FLAG_* bits."""
+    flags = ctypes.c_uint32(0)
+    st = load_library().ffd_check_device_status(_ptr(workspace), ctypes.byref(flags),
+                                                _stream(stream))
+    if st not in (FFD_OK, FFD_ERR_DEVICE_CHECK):
+        raise FFDError(st, "ffd_check_device_status")
+    return int(flags.value)
+
+
+class DecodeBuffers:
+    """Device buffers one decode step needs besides the caller's KV cache.
+
+    Allocation is PyTorch's job (caching allocator); the library only
+    receives pointers.
+    """
+
+    def __init__(self, shape: Shape, device="cuda"):
+        import torch
+        self.shape = shape
+        B, Hq, Hkv = shape.batch, shape.num_q_heads, shape.num_kv_heads
+        cap, T, D = shape.capacity, shape.block_size, shape.head_dim
+        self.k_packed = torch.empty((B, Hkv, cap, D // 2), dtype=torch.uint8, device=device)
+        self.k_scales = torch.empty((B, Hkv, cap // T, D), dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
+        self.mask = torch.empty((B, Hkv, math.ceil(cap // T / 32)), dtype=torch.int32,
+                                device=device)
+        ws = decode_workspace_bytes(shape)
+        self.workspace = torch.empty((max(ws, 256) + 15) // 16 * 16, dtype=torch.uint8,
+                                     device=device)
+        workspace_init(shape, self.workspace)

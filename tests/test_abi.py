@@ -1,0 +1,132 @@
+"""Boundary checks that need no GPU: the library loads, exports every entry
+point the header declares, sizes its buffers correctly, and rejects bad
+arguments on the host before any launch."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_long_context_ffd_b200 import ffd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ffd.h")
+PKG = os.path.join(ROOT, "sparse_long_context_ffd_b200")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ffd_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = ffd.load_library()
+    declared = _declared_functions()
+    assert sorted(ffd.EXPORTED) == declared
+    out = subprocess.run(["nm", "-D", "--defined-only", ffd.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (ffd_\w+)", out))
+    assert set(declared) <= exported
+    for name in declared:
+        assert getattr(lib, name) is not None
+
+
+def test_build_targets_sm100a():
+    from sparse_long_context_ffd_b200 import build
+    assert build.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert "--use_fast_math" not in build.NVCC_FLAGS  # the selector needs IEEE fp32
+
+
+def test_abi_version_and_status_strings():
+    assert ffd.abi_version() == 1
+    assert ffd.status_string(ffd.FFD_OK) == "ok"
+    for code in range(1, 7):
+        assert ffd.status_string(code) not in ("ok", "unknown status")
+    assert ffd.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,cap,T,S", [
+    (1, 4, 1, 4096, 64, 16), (4, 32, 8, 32768, 64, 32), (1, 32, 8, 131072, 64, 64),
+    (1, 32, 8, 262144, 128, 64), (16, 32, 8, 65536, 64, 32), (3, 8, 8, 640, 64, 3)])
+def test_buffer_sizes(B, Hq, Hkv, cap, T, S):
+    s = ffd.make_shape(B, Hq, Hkv, cap, T, S)
+    assert ffd.packed_bytes(s) == B * Hkv * cap * 64
+    assert ffd.scale_bytes(s) == B * Hkv * (cap // T) * 128 * 2
+    assert ffd.mask_words(s) == B * Hkv * math.ceil(cap // T / 32)
+    nsplit = math.ceil(cap // T / S)
+    partials = B * Hkv * nsplit * (Hq // Hkv) * 132 * 4
+    ws = ffd.decode_workspace_bytes(s)
+    assert ws >= partials + B * Hkv * 4 + 4 and ws % 256 == 0
+    assert ws <= partials + 4 * 256 + B * Hkv * 4 + B * Hkv * nsplit * math.ceil(S / 32) * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, ffd.FFD_ERR_UNSUPPORTED), ("head_dim", 0, ffd.FFD_ERR_INVALID_ARG),
+    ("block_size", 32, ffd.FFD_ERR_UNSUPPORTED), ("block_size", -1, ffd.FFD_ERR_INVALID_ARG),
+    ("capacity", 4000, ffd.FFD_ERR_INVALID_ARG), ("capacity", -64, ffd.FFD_ERR_INVALID_ARG),
+    ("split_blocks", 0, ffd.FFD_ERR_INVALID_ARG), ("split_blocks", 513, ffd.FFD_ERR_UNSUPPORTED),
+    ("num_q_heads", 12, ffd.FFD_ERR_UNSUPPORTED), ("num_q_heads", 6, ffd.FFD_ERR_INVALID_ARG),
+    ("num_kv_heads", 0, ffd.FFD_ERR_INVALID_ARG), ("batch", -1, ffd.FFD_ERR_INVALID_ARG),
+])
+def test_bad_shapes_rejected_on_host(field, value, status):
+    s = ffd.make_shape(2, 16, 4, 4096, 64, 16)
+    setattr(s, field, value)
+    lib = ffd.load_library()
+    assert ffd.packed_bytes(s) == 0 and ffd.decode_workspace_bytes(s) == 0
+    fake = 1 << 20  # never dereferenced: the shape check fails first
+    rc = lib.ffd_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 1.0, fake, fake, fake,
+                        1 << 30, None)
+    assert rc == status
+    rc = lib.ffd_quantize_keys(ctypes.byref(s), fake, fake, 0, fake, fake, None)
+    assert rc == status
+
+
+def test_bad_arguments_rejected_on_host():
+    lib = ffd.load_library()
+    s = ffd.make_shape(2, 16, 4, 4096, 64, 16)
+    ws = ffd.decode_workspace_bytes(s)
+    a = 1 << 20  # 16-byte aligned, never dereferenced on these paths
+
+    def dec(q=a, k=a, v=a, p=a, sc=a, ln=a, delta=1.0, out=a, mask=a, w=a, wb=ws):
+        return lib.ffd_decode(ctypes.byref(s), q, k, v, p, sc, ln, delta, out, mask, w, wb, None)
+
+    assert dec(delta=float("nan")) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(delta=-0.5) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(w=None) == ffd.FFD_ERR_WORKSPACE
+    assert dec(wb=ws - 1) == ffd.FFD_ERR_WORKSPACE
+    for name in ("q", "k", "v", "ln", "out", "mask"):
+        assert dec(**{name: None}) == ffd.FFD_ERR_INVALID_ARG, name
+        assert dec(**{name: a + 2}) == ffd.FFD_ERR_INVALID_ARG, name
+    assert dec(p=None) == ffd.FFD_ERR_INVALID_ARG  # the scan needs the packed keys
+    assert dec(sc=a + 8) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_quantize_keys(ctypes.byref(s), a, a, -2, a, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_quantize_keys(ctypes.byref(s), None, a, 0, a, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_quantize_keys(ctypes.byref(s), a, a, 0, a + 4, a, None) == ffd.FFD_ERR_INVALID_ARG
+    # block_begin past the last block and an empty batch are no-ops
+    assert lib.ffd_quantize_keys(ctypes.byref(s), a, a, 64, a, a, None) == ffd.FFD_OK
+    s0 = ffd.make_shape(0, 16, 4, 4096, 64, 16)
+    assert lib.ffd_quantize_keys(ctypes.byref(s0), None, None, 0, None, None, None) == ffd.FFD_OK
+    assert lib.ffd_decode(ctypes.byref(s0), None, None, None, None, None, None, 1.0, None, None,
+                          a, 1 << 20, None) == ffd.FFD_OK
+    assert lib.ffd_workspace_init(ctypes.byref(s), a, ws - 1, None) == ffd.FFD_ERR_WORKSPACE
+    assert lib.ffd_check_device_status(None, None, None) == ffd.FFD_ERR_INVALID_ARG
+
+
+def test_product_path_never_touches_the_oracle():
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
+                assert "ffd_oracle" not in text and "ffdo_" not in text, f
+
+
+def test_binding_has_no_cpu_fallback():
+    import torch
+    s = ffd.make_shape(1, 4, 1, 128, 64, 2)
+    t = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        ffd.decode(s, t, t, t, t, t, t, 1.0, t, t, t)
