@@ -506,6 +506,22 @@ def run_reference(args):
 
 # ------------------------------------------------------------------- main --
 
+def run_profile(args):
+    """A few eager steps on one GPU and nothing else: the target for ncu."""
+    import torch
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = fw.WORKLOADS[args.workload]
+    delta = w.delta if args.delta is None else args.delta
+    inp = fw.make_inputs(w)
+    rep = Replica(w, inp, device, 1)
+    for i in range(args.profile_steps):
+        rep.step(i, delta)
+    torch.cuda.synchronize(device)
+    rep.check_flags()
+    print(f"profile: {args.profile_steps} eager steps of {w.name} (delta {delta}) done")
+    return 0
+
+
 def run_gpu(args):
     import torch
     rank, local_rank, world = dist_env()
@@ -633,11 +649,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--reference-budget", type=float, default=150.0)
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run this many eager steps and exit (for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_steps:
+        return run_profile(args)
     return run_gpu(args)
 
 
