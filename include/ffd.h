@@ -143,6 +143,29 @@ ffd_status ffd_decode(const ffd_shape *shape, const void *q_bf16, const void *k_
                       const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                       void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* ffd_decode without a caller workspace, for callers that cannot allocate
+ * device memory: e.g. a plug-in inside an inference engine that is given only
+ * its input and output buffers, or a serving loop that must not call
+ * cudaMalloc once running (an allocation can synchronise the whole device).
+ * The paper has no counterpart to this entry point; it is a deployment aid.
+ *
+ * Same arguments and results as ffd_decode, minus the workspace.  The kernel's
+ * scratch lives in a fixed 16 MiB device array inside this library, held on
+ * every GPU that loads the library until the process exits; this call
+ * allocates nothing.  Shapes whose ffd_decode_workspace_bytes exceeds
+ * 16 MiB (16777216 bytes) return FFD_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it, so make that first call before any stream
+ * capture.  Every call clears the array's counters and error word on the
+ * stream first; the array is shared by all calls on a device and keeps the
+ * last call's contents, so calls that overlap on the GPU race and must be
+ * serialised by the caller.  Device-side length errors still yield zero rows
+ * and an empty mask, but there is no workspace from which to read the flag. */
+ffd_status ffd_decode_no_alloc(const ffd_shape *shape, const void *q_bf16, const void *k_bf16,
+                               const void *v_bf16, const void *k_packed, const void *k_scales,
+                               const int32_t *d_lengths, float delta, void *out_bf16,
+                               uint32_t *mask, void *cuda_stream);
+
 /* Synchronise the stream, read and clear the workspace's sticky device error
  * word.  *flags_out (may be NULL) receives FFD_DEVICE_FLAG_* bits.  Returns
  * FFD_ERR_DEVICE_CHECK if any flag was set, FFD_ERR_CUDA on a CUDA error. */
