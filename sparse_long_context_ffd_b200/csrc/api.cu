@@ -53,14 +53,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// K or V cache viewed as rows of 128 bf16 (256 bytes); 64 x 64 boxes with
-// the 128-byte swizzle (one box = one 64-channel half of a 64-token tile).
+// K or V cache viewed as rows of 128 bf16 (256 bytes); boxes of 64 channels
+// x kKvBoxRows tokens with the 128-byte swizzle (one box = one 64-channel
+// half of an attention pipeline stage).
 bool make_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), rows > 0 ? rows : 1};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kKvBoxRows)};
   const cuuint32_t elem_strides[2] = {1, 1};
   const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                             strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,

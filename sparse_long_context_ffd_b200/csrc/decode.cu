@@ -5,28 +5,28 @@
 // Kernel and System Optimization"): a selector streams the low-bit keys,
 // computes tentative block scores and filters blocks against a threshold; the
 // computer fetches full-precision K/V only for the kept blocks and computes
-// exact attention.  The threshold is delta below a running maximum inside a
+// exact attention, reusing the scan's decision without a memory round trip
+// (arXiv abstract).  The threshold is delta below a running maximum inside a
 // fixed split of blocks (Methodology 2, Mechanism), so splits never wait for
 // one another; splits are merged with log-sum-exp (flash-decoding split-K).
 //
-// One CTA per work unit (split s, kv-head g, sequence b), 4 consumer warps +
-// 1 producer warp:
-//   phase 1 (selector, skipped when dense): the producer streams the split's
-//     packed-key tiles and scales with 1-D bulk copies into a ring of shared
-//     memory stages; each consumer warp folds the query group into int8 for
-//     one block, runs the integer dot products on the tensor cores
-//     (mma m16n8k32, u8 nibbles x s8 query) and keeps the block maximum.
-//   phase 2: warp 0 turns the block scores into keep bits with a warp-wide
-//     prefix maximum per head and the union over the group (no HBM traffic:
-//     the scan's decision stays on chip).
-//   phase 3 (computer): the producer fetches the kept blocks' K and V in
-//     64-token stages with 2-D TMA copies (128-byte swizzle); each consumer
-//     warp owns 16 tokens of every stage, runs q.K^T and P.V on the tensor
-//     cores (mma m16n8k16 bf16, the query group as the M dimension) with an
-//     online softmax in base 2.
-//   phase 4: the warps' partial softmax states are merged in shared memory
-//     and written as the split partial; the last CTA to finish for (b, g)
-//     merges all splits, writes the bf16 output rows and the mask row.
+// One CTA per work unit (split s, kv-head g, sequence b); three warp roles
+// run concurrently as a pipeline:
+//   producer warp (one lane): an event loop that streams the split's packed
+//     key tiles and scales into the scan ring with 1-D bulk copies and, as
+//     kept blocks appear in the selection queue, their K and V into the
+//     attention ring with 2-D TMA copies (128-byte swizzle);
+//   scan warp: folds the query group into int8 for each block, scores all
+//     tokens on the tensor cores (mma m16n8k32, u8 nibbles x s8 query), keeps
+//     the per-head running maximum in registers, applies the Top-delta test,
+//     takes the union over the group and appends kept blocks to the queue --
+//     the decision never leaves shared memory;
+//   attention warps: each takes whole K/V stages round-robin and runs
+//     S^T = K Q^T (tokens as the mma M dimension), an online softmax in base 2
+//     and O^T += V^T P^T on the tensor cores (mma m16n8k16 bf16).
+// At the end the attention warps merge their softmax states, write the split
+// partial, and the last CTA to finish for (b, g) merges all splits and writes
+// the bf16 output rows and the mask row.  No CTA ever waits for another.
 #include <cuda_bf16.h>
 
 #include <atomic>
@@ -43,35 +43,76 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr float kRsqrtD = 0.08838834764831845f;     // nearest float to 1/sqrt(128)
 constexpr float kScaleLog2 = 0.12751743074195287f;  // log2(e) / sqrt(128)
 
+// Pipeline geometry.
+constexpr int kAttnWarps = 4;
+constexpr int kScanWarp = kAttnWarps;
+constexpr int kProducerWarp = kAttnWarps + 1;
+constexpr int kThreads = (kAttnWarps + 2) * 32;
+constexpr int kAttnThreads = kAttnWarps * 32;
+constexpr int kKvTok = kKvBoxRows;                  // tokens per attention stage
+constexpr int kKvHalfBytes = kKvTok * 128;          // one 64-channel half of K or V
+constexpr int kKvStageBytes = 4 * kKvHalfBytes;     // K lo, K hi, V lo, V hi: 16 KiB
+constexpr int kKvStagesN = 5;
+constexpr int kKvRingBytes = kKvStagesN * kKvStageBytes;
+constexpr int kMergeBytes = kAttnWarps * (8 + 8 + 8 * kHeadDim) * 4;
+
 template <int T>
 struct ScanGeom {
   static constexpr int kStageBytes = T * kPackedRowBytes + kScaleRowBytes;
-  static constexpr int kStages = kRingBytes / kStageBytes;
+  static constexpr int kStages = T == 64 ? 4 : 2;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
+};
+
+template <int T>
+struct SmemLayout {
+  static constexpr int kKvRing = 0;
+  static constexpr int kScanRing = kKvRingBytes;
+  static constexpr int kBars = kScanRing + ScanGeom<T>::kRingBytes;
+  static constexpr int kNumBars = 2 * ScanGeom<T>::kStages + 2 * kKvStagesN;
+  static constexpr int kMeta = kBars + 8 * kNumBars;     // int [kKvStagesN] token offsets
+  static constexpr int kSeq = kMeta + 4 * kKvStagesN;    // int [kKvStagesN] item indices
+  static constexpr int kCtrl = kSeq + 4 * kKvStagesN;    // qcount, sel_done, is_last, abort
+  static constexpr int kKeep = kCtrl + 16;               // u32 [split_words]
+  // queue of kept block indices (u16 [split_blocks]) follows keep bits
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ int clamp127(int x) { return min(127, max(-127, x)); }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat162 v) {
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void raise_timeout(const DecodeParams &p, volatile int *flags) {
-  flags[1] = 1;
+__device__ __forceinline__ void raise_timeout(const DecodeParams &p, volatile int *ctrl) {
+  ctrl[3] = 1;
   atomicOr(p.err, kFlagTimeout);
 }
 
+// Spin (bounded) until the producer has published item `it` in a stage.
+__device__ __forceinline__ bool wait_item_published(volatile int *seq, int st, int it) {
+  if (seq[st] == it) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (seq[st] != it) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(20);
+  }
+  return true;
+}
+
 // Wait for the most recent fill of each ring stage (bounded), so that no
-// bulk copy is still writing this CTA's shared memory when it exits.
+// copy is still writing this CTA's shared memory when it exits.
 __device__ __forceinline__ void drain_ring(uint64_t *full, int stages, int issued) {
   for (int u = issued > stages ? issued - stages : 0; u < issued; ++u)
     mbar_wait(&full[u % stages], static_cast<uint32_t>(u / stages) & 1u, kWaitLimitNs);
 }
 
-// Selector for one block: fold the group's query with the block's channel
-// scales into int8, integer-score every token on the tensor cores, and
-// write score_j for each head of the group.
+// Selector for one block (executed by one warp): fold the group's query with
+// the block's channel scales into int8, integer-score every token on the
+// tensor cores and return, in lane (0, t4), the scores of heads 2*t4 and
+// 2*t4 + 1.
 //
 // Lane (gid = lane / 4, t4 = lane % 4) folds head gid over channels
 // 32*t4 .. 32*t4 + 31, which are exactly the channels its mma B fragments
@@ -81,7 +122,7 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int stages, int issue
 template <int T, int G>
 __device__ __forceinline__ void scan_block(const uint8_t *tile, const uint16_t *scl,
                                            const uint32_t (&qreg)[16], int valid_rows, int lane,
-                                           float *score_out) {
+                                           float &score0, float &score1) {
   const int gid = lane >> 2, t4 = lane & 3;
   float pc[32];
   float a = 0.0f;
@@ -164,35 +205,35 @@ __device__ __forceinline__ void scan_block(const uint8_t *tile, const uint16_t *
   const int sq1 = __shfl_sync(kFull, sumq, h1 << 2);
   const float c0 = __shfl_sync(kFull, cf, h0 << 2);
   const float c1 = __shfl_sync(kFull, cf, h1 << 2);
-  if (gid == 0) {
-    if (h0 < G) score_out[h0] = __fmul_rn(__int2float_rn(best0 - 8 * sq0), c0);
-    if (h1 < G) score_out[h1] = __fmul_rn(__int2float_rn(best1 - 8 * sq1), c1);
-  }
-}
-
-// Byte address of 16-byte chunk `cc` (0..15) of row `r` in a K or V stage
-// tile: two 64-channel halves of 64 rows x 128 bytes, 128-byte swizzled.
-__device__ __forceinline__ uint32_t kv_chunk_addr(uint32_t base, int r, int cc) {
-  return base + static_cast<uint32_t>((cc >> 3) * 8192 + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
+  score0 = __fmul_rn(__int2float_rn(best0 - 8 * sq0), c0);
+  score1 = __fmul_rn(__int2float_rn(best1 - 8 * sq1), c1);
 }
 
 template <int T, int G>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
-  constexpr int NS1 = ScanGeom<T>::kStages;
-  constexpr int kScanStage = ScanGeom<T>::kStageBytes;
+  using SG = ScanGeom<T>;
+  using SL = SmemLayout<T>;
+  constexpr int NSA = SG::kStages;
+  constexpr int kSubPerBlock = T / kKvTok;
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *ring = smem;
-  uint64_t *full1 = reinterpret_cast<uint64_t *>(smem + kRingBytes);
-  uint64_t *empty1 = full1 + NS1;
-  uint64_t *full3 = empty1 + NS1;
-  uint64_t *empty3 = full3 + kKvStages;
-  volatile int *flags = reinterpret_cast<volatile int *>(empty3 + kKvStages);  // is_last, abort
-  uint32_t *keepbits = reinterpret_cast<uint32_t *>(empty3 + kKvStages) + 4;
-  float *scores = reinterpret_cast<float *>(keepbits + ((p.split_words + 3) & ~3));
+  uint8_t *kv_ring = smem + SL::kKvRing;
+  uint8_t *scan_ring = smem + SL::kScanRing;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SL::kBars);
+  uint64_t *full_a = bars;
+  uint64_t *empty_a = full_a + NSA;
+  uint64_t *full_b = empty_a + NSA;
+  uint64_t *empty_b = full_b + kKvStagesN;
+  volatile int *meta = reinterpret_cast<volatile int *>(smem + SL::kMeta);
+  volatile int *seq = reinterpret_cast<volatile int *>(smem + SL::kSeq);
+  volatile int *ctrl = reinterpret_cast<volatile int *>(smem + SL::kCtrl);  // qcount, done, last, abort
+  uint32_t *keepbits = reinterpret_cast<uint32_t *>(smem + SL::kKeep);
+  volatile uint16_t *queue =
+      reinterpret_cast<volatile uint16_t *>(keepbits + ((p.split_words + 3) & ~3));
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,7 +243,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
   const int nb = bad ? 0 : (len + T - 1) / T;
   const int nsplit = (nb + p.split_blocks - 1) / p.split_blocks;
   const size_t row = static_cast<size_t>(b) * p.num_kv_heads + g;
-  uint16_t *out_rows = p.out + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim;
+  uint16_t *out_rows =
+      p.out + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim;
 
   if (split >= nsplit) {
     // Empty or invalid sequence: split 0 writes zero rows and an empty mask.
@@ -218,294 +260,351 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
   const bool dense = p.dense != 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS1; ++s) {
-      mbar_init(&full1[s], 1);
-      mbar_init(&empty1[s], 1);
+    for (int s = 0; s < NSA; ++s) {
+      mbar_init(&full_a[s], 1);
+      mbar_init(&empty_a[s], 1);
     }
-    for (int s = 0; s < kKvStages; ++s) {
-      mbar_init(&full3[s], 1);
-      mbar_init(&empty3[s], kConsumerWarps);
+    for (int s = 0; s < kKvStagesN; ++s) {
+      mbar_init(&full_b[s], 1);
+      mbar_init(&empty_b[s], 1);
+      seq[s] = -1;
     }
-    flags[0] = 0;
-    flags[1] = 0;
+    ctrl[0] = 0;
+    ctrl[1] = 0;
+    ctrl[2] = 0;
+    ctrl[3] = 0;
     fence_mbar_init();
   }
-  if (warp == kConsumerWarps && lane == 0) {
+  for (int w = threadIdx.x; w < p.split_words; w += blockDim.x) keepbits[w] = 0u;
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
   __syncthreads();
 
-  // ---------------------------------------------------------- phase 1: scan
-  if (!dense) {
-    if (warp == kConsumerWarps) {
-      if (lane == 0) {
-        const uint8_t *src_p =
-            p.packed + (row * p.capacity + static_cast<size_t>(j0) * T) * kPackedRowBytes;
-        const uint16_t *src_s =
-            p.scales + (row * static_cast<size_t>(p.capacity / T) + j0) * kHeadDim;
-        int i = 0;
-        for (; i < nbs; ++i) {
-          const int st = i % NS1;
-          const uint32_t use = static_cast<uint32_t>(i / NS1);
-          if (use > 0 && !mbar_wait(&empty1[st], (use - 1) & 1u, kWaitLimitNs)) {
-            raise_timeout(p, flags);
-            break;
-          }
-          uint8_t *dst = ring + st * kScanStage;
-          mbar_arrive_expect_tx(&full1[st], kScanStage);
-          bulk_g2s(dst, src_p + static_cast<size_t>(i) * T * kPackedRowBytes, T * kPackedRowBytes,
-                   &full1[st]);
-          bulk_g2s(dst + T * kPackedRowBytes, src_s + static_cast<size_t>(i) * kHeadDim,
-                   kScaleRowBytes, &full1[st]);
-          if (flags[1]) {
-            ++i;
-            break;
-          }
-        }
-        drain_ring(full1, NS1, i);
+  // ================================================================ producer
+  if (warp == kProducerWarp) {
+    if (lane != 0) return;
+    const uint8_t *src_p =
+        p.packed + (row * p.capacity + static_cast<size_t>(j0) * T) * kPackedRowBytes;
+    const uint16_t *src_s = p.scales + (row * static_cast<size_t>(p.capacity / T) + j0) * kHeadDim;
+    const int row_tok0 = static_cast<int>(row * p.capacity);
+    const int scan_total = dense ? 0 : nbs;
+    int sc_next = 0;                // scan tiles issued
+    int it_next = 0;                // attention stages issued (items + end markers)
+    int q_ptr = 0, sub = 0;         // position in the kept-block list
+    int ends_sent = 0;
+    uint64_t idle_since = 0;
+    while (true) {
+      bool progress = false;
+      // scan tiles
+      while (sc_next < scan_total) {
+        const int st = sc_next % NSA;
+        const int use = sc_next / NSA;
+        if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
+        uint8_t *dst = scan_ring + st * SG::kStageBytes;
+        mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
+        bulk_g2s(dst, src_p + static_cast<size_t>(sc_next) * T * kPackedRowBytes,
+                 T * kPackedRowBytes, &full_a[st]);
+        bulk_g2s(dst + T * kPackedRowBytes, src_s + static_cast<size_t>(sc_next) * kHeadDim,
+                 kScaleRowBytes, &full_a[st]);
+        ++sc_next;
+        progress = true;
       }
-    } else {
-      const int gid = lane >> 2, t4 = lane & 3;
-      uint32_t qreg[16];
-      if (gid < G) {
-        const uint4 *qsrc = reinterpret_cast<const uint4 *>(
-            p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid) * kHeadDim +
-            32 * t4);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = qsrc[v];
-          qreg[4 * v] = x.x;
-          qreg[4 * v + 1] = x.y;
-          qreg[4 * v + 2] = x.z;
-          qreg[4 * v + 3] = x.w;
+      // K/V stages for the kept blocks published so far
+      const bool sel_done = dense || ctrl[1] != 0;
+      __threadfence_block();
+      const int avail = dense ? nbs : ctrl[0];
+      while (q_ptr < avail) {
+        const int j = dense ? q_ptr : static_cast<int>(queue[q_ptr]);
+        const int tok = (j0 + j) * T + sub * kKvTok;
+        if (sub >= kSubPerBlock || tok >= len) {
+          ++q_ptr;
+          sub = 0;
+          continue;
         }
+        const int st = it_next % kKvStagesN;
+        const int use = it_next / kKvStagesN;
+        if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
+        uint8_t *dst = kv_ring + st * kKvStageBytes;
+        meta[st] = tok;
+        seq[st] = it_next;
+        mbar_arrive_expect_tx(&full_b[st], kKvStageBytes);
+        const int y = row_tok0 + tok;
+        tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);
+        tma_load_2d(dst + kKvHalfBytes, &tmap_k, 64, y, &full_b[st]);
+        tma_load_2d(dst + 2 * kKvHalfBytes, &tmap_v, 0, y, &full_b[st]);
+        tma_load_2d(dst + 3 * kKvHalfBytes, &tmap_v, 64, y, &full_b[st]);
+        ++it_next;
+        ++sub;
+        progress = true;
+      }
+      // once the selection is complete and every kept stage is issued, one
+      // end marker per attention warp
+      if (sel_done && q_ptr >= avail) {
+        while (ends_sent < kAttnWarps) {
+          const int st = it_next % kKvStagesN;
+          const int use = it_next / kKvStagesN;
+          if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
+          meta[st] = -1;
+          seq[st] = it_next;
+          mbar_arrive(&full_b[st]);
+          ++it_next;
+          ++ends_sent;
+          progress = true;
+        }
+        if (ends_sent == kAttnWarps) break;
+      }
+      if (ctrl[3]) break;
+      if (progress) {
+        idle_since = 0;
       } else {
-#pragma unroll
-        for (int v = 0; v < 16; ++v) qreg[v] = 0u;
-      }
-      for (int i = warp; i < nbs; i += kConsumerWarps) {
-        const int st = i % NS1;
-        const uint32_t use = static_cast<uint32_t>(i / NS1);
-        if (!mbar_wait(&full1[st], use & 1u, kWaitLimitNs)) {
-          raise_timeout(p, flags);
+        const uint64_t now = global_timer_ns();
+        if (idle_since == 0) {
+          idle_since = now;
+        } else if (now - idle_since > kWaitLimitNs) {
+          raise_timeout(p, ctrl);
           break;
         }
-        const uint8_t *tile = ring + st * kScanStage;
-        scan_block<T, G>(tile, reinterpret_cast<const uint16_t *>(tile + T * kPackedRowBytes), qreg,
-                         min(T, len - (j0 + i) * T), lane, scores + i * G);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty1[st]);
-        if (flags[1]) break;
+        __nanosleep(32);
       }
     }
+    drain_ring(full_a, NSA, sc_next);
+    drain_ring(full_b, kKvStagesN, it_next);
+    return;
   }
-  fence_proxy_async_smem();  // generic reads of the ring before TMA reuses it
-  __syncthreads();
 
-  // ------------------------------------------- phase 2: Top-delta keep bits
-  if (warp == 0) {
-    float carry[G];
+  // ============================================================ scan warp
+  if (warp == kScanWarp) {
+    if (dense) return;
+    const int gid = lane >> 2, t4 = lane & 3;
+    uint32_t qreg[16];
+    if (gid < G) {
+      const uint4 *qsrc = reinterpret_cast<const uint4 *>(
+          p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid) * kHeadDim +
+          32 * t4);
 #pragma unroll
-    for (int h = 0; h < G; ++h) carry[h] = -INFINITY;
-    for (int base = 0; base < nbs; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < nbs;
-      bool keep = dense && valid;
-      if (!dense) {
+      for (int v = 0; v < 4; ++v) {
+        const uint4 x = qsrc[v];
+        qreg[4 * v] = x.x;
+        qreg[4 * v + 1] = x.y;
+        qreg[4 * v + 2] = x.z;
+        qreg[4 * v + 3] = x.w;
+      }
+    } else {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float s = valid ? scores[i * G + h] : -INFINITY;
-          float m = s;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float o = __shfl_up_sync(kFull, m, off);
-            if (lane >= off) m = fmaxf(m, o);
-          }
-          m = fmaxf(m, carry[h]);
-          carry[h] = __shfl_sync(kFull, m, 31);
-          keep = keep || (valid && s >= __fsub_rn(m, p.delta));
+      for (int v = 0; v < 16; ++v) qreg[v] = 0u;
+    }
+    float run0 = -INFINITY, run1 = -INFINITY;  // running max of heads 2*t4, 2*t4 + 1
+    int qn = 0;
+    for (int i = 0; i < nbs; ++i) {
+      const int st = i % NSA;
+      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(i / NSA) & 1u, kWaitLimitNs)) {
+        raise_timeout(p, ctrl);
+        break;
+      }
+      const uint8_t *tile = scan_ring + st * SG::kStageBytes;
+      float s0, s1;
+      scan_block<T, G>(tile, reinterpret_cast<const uint16_t *>(tile + T * kPackedRowBytes), qreg,
+                       min(T, len - (j0 + i) * T), lane, s0, s1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_a[st]);
+      // Top-delta against the running maximum of the split, union over the group
+      bool keep = false;
+      if (gid == 0) {
+        if (2 * t4 < G) {
+          run0 = fmaxf(run0, s0);
+          keep = s0 >= __fsub_rn(run0, p.delta);
+        }
+        if (2 * t4 + 1 < G) {
+          run1 = fmaxf(run1, s1);
+          keep = keep || (s1 >= __fsub_rn(run1, p.delta));
         }
       }
-      const uint32_t bits = __ballot_sync(kFull, keep);
-      if (lane == 0) keepbits[base >> 5] = bits;
+      if (__any_sync(kFull, keep)) {
+        if (lane == 0) {
+          keepbits[i >> 5] |= 1u << (i & 31);
+          queue[qn] = static_cast<uint16_t>(i);
+          __threadfence_block();
+          ctrl[0] = qn + 1;
+        }
+        ++qn;
+      }
+      if (ctrl[3]) break;
     }
-  }
-  __syncthreads();
-
-  // ------------------------------------------- phase 3: attention (computer)
-  if (warp == kConsumerWarps) {
     if (lane == 0) {
-      int it = 0;
-      bool ok = flags[1] == 0;
-      for (int w = 0; ok && w < p.split_words; ++w) {
-        uint32_t bits = keepbits[w];
-        while (ok && bits) {
-          const int i = 32 * w + __ffs(bits) - 1;
-          bits &= bits - 1;
-#pragma unroll 1
-          for (int u = 0; u < T / kSubTokens; ++u) {
-            const int tok = (j0 + i) * T + u * kSubTokens;
-            if (tok >= len) break;
-            const int st = it % kKvStages;
-            const uint32_t use = static_cast<uint32_t>(it / kKvStages);
-            if (use > 0 && !mbar_wait(&empty3[st], (use - 1) & 1u, kWaitLimitNs)) {
-              raise_timeout(p, flags);
-              ok = false;
-              break;
-            }
-            uint8_t *dst = ring + st * kKvStageBytes;
-            mbar_arrive_expect_tx(&full3[st], kKvStageBytes);
-            const int y = static_cast<int>(row * p.capacity) + tok;
-            tma_load_2d(dst, &tmap_k, 0, y, &full3[st]);
-            tma_load_2d(dst + 8192, &tmap_k, 64, y, &full3[st]);
-            tma_load_2d(dst + 16384, &tmap_v, 0, y, &full3[st]);
-            tma_load_2d(dst + 24576, &tmap_v, 64, y, &full3[st]);
-            ++it;
-          }
-        }
-      }
-      drain_ring(full3, kKvStages, it);
+      __threadfence_block();
+      ctrl[1] = 1;
     }
     return;
   }
 
+  // ======================================================= attention warps
   const int gid = lane >> 2, t4 = lane & 3;
-  uint32_t qa[8][2];
+  // Q^T as the mma B operand: k-step ks holds channels 16ks + 2*t4 (+1) and
+  // 16ks + 8 + 2*t4 (+1) of head gid.
+  uint32_t qb[8][2];
   {
     const uint32_t *qh = reinterpret_cast<const uint32_t *>(
         p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + (gid < G ? gid : 0)) *
                   kHeadDim);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      qa[s][0] = gid < G ? qh[8 * s + t4] : 0u;      // channels 16s + 2*t4, +1
-      qa[s][1] = gid < G ? qh[8 * s + 4 + t4] : 0u;  // channels 16s + 8 + 2*t4, +1
+    for (int ks = 0; ks < 8; ++ks) {
+      qb[ks][0] = gid < G ? qh[8 * ks + t4] : 0u;
+      qb[ks][1] = gid < G ? qh[8 * ks + 4 + t4] : 0u;
     }
   }
-  float m_run = -INFINITY, l_run = 0.0f;
-  float acc[16][4];
+  float m_run[2] = {-INFINITY, -INFINITY};  // heads 2*t4, 2*t4 + 1
+  float l_run[2] = {0.0f, 0.0f};
+  float oacc[8][4];  // O^T: channel tile cm, rows 16cm + gid (+8), heads 2*t4 (+1)
 #pragma unroll
-  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+  for (int cm = 0; cm < 8; ++cm) oacc[cm][0] = oacc[cm][1] = oacc[cm][2] = oacc[cm][3] = 0.0f;
 
-  const uint32_t ring_addr = smem_addr(ring);
-  int it = 0;
-  bool ok = flags[1] == 0;
-  for (int w = 0; ok && w < p.split_words; ++w) {
-    uint32_t bits = keepbits[w];
-    while (ok && bits) {
-      const int i = 32 * w + __ffs(bits) - 1;
-      bits &= bits - 1;
-#pragma unroll 1
-      for (int u = 0; u < T / kSubTokens; ++u) {
-        const int tok = (j0 + i) * T + u * kSubTokens;
-        if (tok >= len) break;
-        const int st = it % kKvStages;
-        const uint32_t use = static_cast<uint32_t>(it / kKvStages);
-        if (!mbar_wait(&full3[st], use & 1u, kWaitLimitNs)) {
-          raise_timeout(p, flags);
-          ok = false;
-          break;
-        }
-        const uint32_t kbase = ring_addr + st * kKvStageBytes;
-        const uint32_t vbase = kbase + 16384;
+  // Per-lane ldmatrix geometry.  K (A operand, non-transposed): row
+  // 16mt + (lane & 7) + 8*((lane >> 3) & 1), 16-byte chunk 2ks + (lane >> 4).
+  // V (A operand of O^T, transposed): row 16mt + (lane & 7) + 8*(lane >> 4),
+  // chunk 2cm + ((lane >> 3) & 1).  Every row index is = lane & 7 (mod 8), so
+  // the 128-byte swizzle XOR is a per-lane constant.
+  const int r7 = lane & 7;
+  const int k_row = r7 + 8 * ((lane >> 3) & 1);
+  const int k_chi = lane >> 4;
+  const int v_row = r7 + 8 * (lane >> 4);
+  const int v_chi = (lane >> 3) & 1;
+  const uint32_t kv_ring_addr = smem_addr(kv_ring);
 
-        // S = Q K^T over this warp's 16 tokens (two n-tiles of 8)
-        float sacc[2][4];
+  for (int it = warp;; it += kAttnWarps) {
+    const int st = it % kKvStagesN;
+    // Items go to the attention warps round-robin, so a warp can reach item
+    // `it` before the stage's previous fill (another warp's item) has landed;
+    // a parity wait could then match that older phase.  The producer writes
+    // `it` into seq[st] only after the previous fill was consumed, so once it
+    // is visible the parity below names exactly this fill.
+    if (!wait_item_published(seq, st, it) ||
+        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / kKvStagesN) & 1u, kWaitLimitNs)) {
+      raise_timeout(p, ctrl);
+      break;
+    }
+    const int tok = meta[st];
+    if (tok < 0) break;
+    const uint32_t kbase = kv_ring_addr + st * kKvStageBytes;
+    const uint32_t vbase = kbase + 2 * kKvHalfBytes;
+
+    // S^T = K Q^T for kKvTok tokens: kKvTok/16 independent accumulator chains
+    constexpr int MT = kKvTok / 16;
+    float sacc[MT][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.0f;
+    for (int mt = 0; mt < MT; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.0f;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+    for (int ks = 0; ks < 8; ++ks) {
+      const int chunk = 2 * ks + k_chi;
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            uint32_t kb[4];
-            ldmatrix_x4(kb, kv_chunk_addr(kbase, 16 * warp + 8 * nt + (lane & 7), 4 * kk + (lane >> 3)));
-            mma_bf16_16x8x16(sacc[nt], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, kb[0], kb[1]);
-            mma_bf16_16x8x16(sacc[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, kb[2], kb[3]);
-          }
-        }
-        // online softmax in base 2; tokens past the length are masked out
-        const int tw = tok + 16 * warp;
-        float x[2][2];
-        float mt = -INFINITY;
+      for (int mt = 0; mt < MT; ++mt) {
+        const int r = 16 * mt + k_row;
+        uint32_t a[4];
+        ldmatrix_x4(a, kbase + (chunk >> 3) * kKvHalfBytes + r * 128 + (((chunk & 7) ^ r7) << 4));
+        mma_bf16_16x8x16(sacc[mt], a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+      }
+    }
+    // online softmax (base 2); tokens at or past the length are masked
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+    for (int mt = 0; mt < MT; ++mt) {
+      const int t_lo = tok + 16 * mt + gid;
+      const bool v_lo = t_lo < len, v_hi = t_lo + 8 < len;
+      sacc[mt][0] = v_lo ? sacc[mt][0] * kScaleLog2 : -INFINITY;
+      sacc[mt][1] = v_lo ? sacc[mt][1] * kScaleLog2 : -INFINITY;
+      sacc[mt][2] = v_hi ? sacc[mt][2] * kScaleLog2 : -INFINITY;
+      sacc[mt][3] = v_hi ? sacc[mt][3] * kScaleLog2 : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(sacc[mt][0], sacc[mt][2]));
+      mx1 = fmaxf(mx1, fmaxf(sacc[mt][1], sacc[mt][3]));
+    }
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = tw + 8 * nt + 2 * t4 + e;
-            x[nt][e] = t < len ? sacc[nt][e] * kScaleLog2 : -INFINITY;
-            mt = fmaxf(mt, x[nt][e]);
-          }
-        }
-        mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 1));
-        mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 2));
-        const float m_new = fmaxf(m_run, mt);
-        float corr = 1.0f;
-        float pv[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};
-        if (m_new != -INFINITY) {
-          corr = exp2f(m_run - m_new);
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float corr0 = mn0 == -INFINITY ? 1.0f : exp2f(m_run[0] - mn0);
+    const float corr1 = mn1 == -INFINITY ? 1.0f : exp2f(m_run[1] - mn1);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    uint32_t pb[MT][2];
+    float ps0 = 0.0f, ps1 = 0.0f;
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
+    for (int mt = 0; mt < MT; ++mt) {
+      const float e0 = mn0 == -INFINITY ? 0.0f : exp2f(sacc[mt][0] - mn0);
+      const float e1 = mn1 == -INFINITY ? 0.0f : exp2f(sacc[mt][1] - mn1);
+      const float e2 = mn0 == -INFINITY ? 0.0f : exp2f(sacc[mt][2] - mn0);
+      const float e3 = mn1 == -INFINITY ? 0.0f : exp2f(sacc[mt][3] - mn1);
+      // P rounded to bf16 once; the same weights feed P.V and the running sum
+      const uint32_t lo = pack_bf16x2(e0, e1);  // token gid, heads 2*t4, 2*t4+1
+      const uint32_t hi = pack_bf16x2(e2, e3);  // token gid + 8
+      ps0 += bf16_lo(lo) + bf16_lo(hi);
+      ps1 += bf16_hi(lo) + bf16_hi(hi);
+      pb[mt][0] = movmatrix_trans(lo);  // head gid, tokens 16mt + 2*t4, +1
+      pb[mt][1] = movmatrix_trans(hi);  // head gid, tokens 16mt + 8 + 2*t4, +1
+    }
+    l_run[0] = l_run[0] * corr0 + ps0;
+    l_run[1] = l_run[1] * corr1 + ps1;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) pv[nt][e] = exp2f(x[nt][e] - m_new);
-        }
-        // P is rounded to bf16 once; the same weights feed P.V and the sum
-        const __nv_bfloat162 p01 = __floats2bfloat162_rn(pv[0][0], pv[0][1]);
-        const __nv_bfloat162 p23 = __floats2bfloat162_rn(pv[1][0], pv[1][1]);
-        const float2 f01 = __bfloat1622float2(p01);
-        const float2 f23 = __bfloat1622float2(p23);
-        l_run = l_run * corr + ((f01.x + f01.y) + (f23.x + f23.y));
+    for (int cm = 0; cm < 8; ++cm) {
+      oacc[cm][0] *= corr0;
+      oacc[cm][1] *= corr1;
+      oacc[cm][2] *= corr0;
+      oacc[cm][3] *= corr1;
+    }
+    // O^T += V^T P^T: 8 channel tiles x kKvTok/16 token steps
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          acc[n][0] *= corr;
-          acc[n][1] *= corr;
-        }
-        const uint32_t pa0 = pack_bf16x2(p01), pa2 = pack_bf16x2(p23);
+    for (int cm = 0; cm < 8; ++cm) {
+      const int chunk = 2 * cm + v_chi;
 #pragma unroll
-        for (int cc2 = 0; cc2 < 8; ++cc2) {
-          const int mi = lane >> 3;
-          uint32_t vb[4];
-          ldmatrix_x4_trans(vb, kv_chunk_addr(vbase, 16 * warp + (lane & 7) + 8 * (mi & 1), 2 * cc2 + (mi >> 1)));
-          mma_bf16_16x8x16(acc[2 * cc2], pa0, 0u, pa2, 0u, vb[0], vb[1]);
-          mma_bf16_16x8x16(acc[2 * cc2 + 1], pa0, 0u, pa2, 0u, vb[2], vb[3]);
-        }
-        m_run = m_new;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty3[st]);
-        ++it;
+      for (int mt = 0; mt < MT; ++mt) {
+        const int r = 16 * mt + v_row;
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vbase + (chunk >> 3) * kKvHalfBytes + r * 128 + (((chunk & 7) ^ r7) << 4));
+        mma_bf16_16x8x16(oacc[cm], a[0], a[1], a[2], a[3], pb[mt][0], pb[mt][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_b[st]);
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l_run[0] += __shfl_xor_sync(kFull, l_run[0], off);
+    l_run[1] += __shfl_xor_sync(kFull, l_run[1], off);
+  }
+
+  // ------------------------------ split partial and the final merge
+  named_barrier(1, kAttnThreads);  // every attention stage consumed; scan ring idle
+  float *wm = reinterpret_cast<float *>(scan_ring);  // [warp][8]
+  float *wl = wm + kAttnWarps * 8;                   // [warp][8]
+  float *wacc = wl + kAttnWarps * 8;                 // [warp][8][128]
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * t4 + e;
+    if (h < G) {
+      if (gid == 0) {
+        wm[warp * 8 + h] = m_run[e];
+        wl[warp * 8 + h] = l_run[e];
+      }
+#pragma unroll
+      for (int cm = 0; cm < 8; ++cm) {
+        wacc[(warp * 8 + h) * kHeadDim + 16 * cm + gid] = oacc[cm][e];
+        wacc[(warp * 8 + h) * kHeadDim + 16 * cm + gid + 8] = oacc[cm][2 + e];
       }
     }
   }
-  l_run += __shfl_xor_sync(kFull, l_run, 1);
-  l_run += __shfl_xor_sync(kFull, l_run, 2);
-
-  // ------------------------------ phase 4: split partial and the final merge
-  const uint32_t nthreads = kConsumerWarps * 32;
-  named_barrier(1, nthreads);  // every stage consumed: the ring becomes scratch
-  float *wm = reinterpret_cast<float *>(ring);  // [warp][8]
-  float *wl = wm + kConsumerWarps * 8;          // [warp][8]
-  float *wacc = wl + kConsumerWarps * 8;        // [warp][8][128]
-  if (gid < G) {
-    if (t4 == 0) {
-      wm[warp * 8 + gid] = m_run;
-      wl[warp * 8 + gid] = l_run;
-    }
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      wacc[(warp * 8 + gid) * kHeadDim + 8 * n + 2 * t4] = acc[n][0];
-      wacc[(warp * 8 + gid) * kHeadDim + 8 * n + 2 * t4 + 1] = acc[n][1];
-    }
-  }
-  named_barrier(1, nthreads);
+  named_barrier(1, kAttnThreads);
   const size_t unit = row * p.nsplit_max + split;
   float *part = p.partials + unit * G * kPartialStride;
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += nthreads) {
+  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAttnThreads) {
     const int h = idx >> 7, c = idx & 127;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, wm[w * 8 + h]);
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, wm[w * 8 + h]);
     float L = 0.0f, A = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < kAttnWarps; ++w) {
       const float mw = wm[w * 8 + h];
       if (mw != -INFINITY) {
         const float f = exp2f(mw - M);
@@ -519,19 +618,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
       part[h * kPartialStride + 129] = L;
     }
   }
-  if (static_cast<int>(threadIdx.x) < p.split_words)
-    p.split_bits[unit * p.split_words + threadIdx.x] = keepbits[threadIdx.x];
+  if (static_cast<int>(threadIdx.x) < p.split_words) {
+    uint32_t bits = keepbits[threadIdx.x];
+    if (dense) {  // every valid block of the split
+      const int lo = 32 * threadIdx.x;
+      bits = lo >= nbs ? 0u : (nbs - lo >= 32 ? kFull : ((1u << (nbs - lo)) - 1u));
+    }
+    p.split_bits[unit * p.split_words + threadIdx.x] = bits;
+  }
   __threadfence();
-  named_barrier(1, nthreads);
+  named_barrier(1, kAttnThreads);
   if (threadIdx.x == 0)
-    flags[0] = atomicAdd(&p.counters[row], 1u) == static_cast<unsigned>(nsplit - 1) ? 1 : 0;
-  named_barrier(1, nthreads);
-  if (!flags[0]) return;
+    ctrl[2] = atomicAdd(&p.counters[row], 1u) == static_cast<unsigned>(nsplit - 1) ? 1 : 0;
+  named_barrier(1, kAttnThreads);
+  if (!ctrl[2]) return;
   __threadfence();
 
   // last CTA of (b, g): log-sum-exp merge over the splits
   const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += nthreads) {
+  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAttnThreads) {
     const int h = idx >> 7, c = idx & 127;
     float M = -INFINITY;
     for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(row_parts + (s * G + h) * kPartialStride + 128));
@@ -545,7 +650,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 2)
     out_rows[h * kHeadDim + c] = __bfloat16_as_ushort(__float2bfloat16_rn(A / L));
   }
   const uint32_t *row_bits = p.split_bits + row * p.nsplit_max * p.split_words;
-  for (int w = threadIdx.x; w < p.mask_words; w += nthreads) {
+  for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads) {
     uint32_t bits = 0;
     for (int k = 0; k < 32; ++k) {
       const int j = 32 * w + k;
@@ -577,7 +682,7 @@ cudaError_t launch_tg(const DecodeParams &p, const CUtensorMap &tk, const CUtens
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  kern<<<grid, kDecodeThreads, smem, stream>>>(p, tk, tv);
+  kern<<<grid, kThreads, smem, stream>>>(p, tk, tv);
   return cudaGetLastError();
 }
 
@@ -593,15 +698,18 @@ cudaError_t launch_t(const DecodeParams &p, const CUtensorMap &tk, const CUtenso
   }
 }
 
+template <int T>
+size_t smem_bytes_t(int split_blocks) {
+  const int split_words = (split_blocks + 31) / 32;
+  return 1024 + SmemLayout<T>::kKeep + 4 * static_cast<size_t>((split_words + 3) & ~3) +
+         2 * static_cast<size_t>((split_blocks + 7) & ~7);
+}
+
 }  // namespace
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks) {
-  const int stage = block_size * kPackedRowBytes + kScaleRowBytes;
-  const int ns1 = kRingBytes / stage;
-  const int split_words = (split_blocks + 31) / 32;
-  return 1024 + kRingBytes + 8 * (2 * ns1 + 2 * kKvStages) + 16 +
-         4 * static_cast<size_t>((split_words + 3) & ~3) +
-         4 * static_cast<size_t>(split_blocks) * group;
+  (void)group;
+  return block_size == 64 ? smem_bytes_t<64>(split_blocks) : smem_bytes_t<128>(split_blocks);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,

@@ -14,15 +14,11 @@ constexpr int kHeadDim = 128;
 constexpr int kPackedRowBytes = kHeadDim / 2;  // 64 bytes of nibbles per token
 constexpr int kScaleRowBytes = kHeadDim * 2;   // 128 bf16 scales per block
 
-// Fused decode kernel geometry.
-constexpr int kConsumerWarps = 4;
-constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kSubTokens = 64;                             // K/V tokens per pipeline stage
-constexpr int kKvStageBytes = 4 * kSubTokens * 64 * 2;     // K lo/hi + V lo/hi halves, 32 KiB
-constexpr int kKvStages = 3;
-constexpr int kRingBytes = kKvStages * kKvStageBytes;  // 96 KiB, reused by the scan
-constexpr int kPartialStride = 132;                    // floats per (split, head): acc[128], m, l
-constexpr uint64_t kWaitLimitNs = 2000000000ull;       // bounded mbarrier waits (2 s)
+// Rows of one TMA box of K or V (tokens per attention pipeline stage); a box
+// is 64 channels (128 bytes, the swizzle span) wide.
+constexpr int kKvBoxRows = 32;
+constexpr int kPartialStride = 132;  // floats per (split, head): acc[128], m, l
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded mbarrier waits (2 s)
 
 constexpr uint32_t kFlagBadLength = 0x1u;
 constexpr uint32_t kFlagTimeout = 0x2u;
