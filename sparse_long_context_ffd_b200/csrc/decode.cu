@@ -634,30 +634,106 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (!ctrl[2]) return;
   __threadfence();
 
-  // last CTA of (b, g): log-sum-exp merge over the splits
+  // last CTA of (b, g): log-sum-exp merge over the splits.  Every load here
+  // is independent of the others, so the merge costs a few L2 round trips
+  // rather than one per split:
+  //   1. per head (one warp per head, lanes striding over the splits):
+  //      M* = max_s m_s and L* = sum_s l_s 2^(m_s - M*);
+  //   2. in chunks of splits: weights 2^(m_s - M*) / L* into shared memory,
+  //      then each thread accumulates four output channels with float4 loads.
   const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAttnThreads) {
-    const int h = idx >> 7, c = idx & 127;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(row_parts + (s * G + h) * kPartialStride + 128));
-    float L = 0.0f, A = 0.0f;
-    for (int s = 0; s < nsplit; ++s) {
+  float *stats = reinterpret_cast<float *>(scan_ring);  // [G][2]: M*, L*
+  float *wts = stats + 16;                              // [chunk][G]
+  for (int h = warp; h < G; h += kAttnWarps) {
+    float m = -INFINITY;
+    for (int s = lane; s < nsplit; s += 32)
+      m = fmaxf(m, __ldcg(row_parts + (s * G + h) * kPartialStride + 128));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+    float l = 0.0f;
+    for (int s = lane; s < nsplit; s += 32) {
       const float *ps = row_parts + (s * G + h) * kPartialStride;
-      const float f = exp2f(__ldcg(ps + 128) - M);
-      L += __ldcg(ps + 129) * f;
-      A += __ldcg(ps + c) * f;
+      l += __ldcg(ps + 129) * exp2f(__ldcg(ps + 128) - m);
     }
-    out_rows[h * kHeadDim + c] = __bfloat16_as_ushort(__float2bfloat16_rn(A / L));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
+    if (lane == 0) {
+      stats[2 * h] = m;
+      stats[2 * h + 1] = l;
+    }
   }
+  named_barrier(1, kAttnThreads);
+  constexpr int kWtsFloats = ScanGeom<T>::kRingBytes / 4 - 16;
+  const int chunk = kWtsFloats / G;
+  const int f = threadIdx.x;  // float4 output index: head f / 32, channels 4 (f % 32) ..
+  float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;  // second set for G == 8
+  for (int s0 = 0; s0 < nsplit; s0 += chunk) {
+    const int cnt = min(chunk, nsplit - s0);
+    for (int i = threadIdx.x; i < cnt * G; i += kAttnThreads) {
+      const int h = i % G, s = s0 + i / G;
+      wts[i] = exp2f(__ldcg(row_parts + (s * G + h) * kPartialStride + 128) - stats[2 * h]) /
+               stats[2 * h + 1];
+    }
+    named_barrier(1, kAttnThreads);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int fi = f + half * kAttnThreads;
+      if (fi < G * 32) {
+        const int h = fi >> 5, c4 = fi & 31;
+        float4 acc = half ? o1 : o0;
+        int s = 0;
+        for (; s + 8 <= cnt; s += 8) {
+          float4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            v[u] = __ldcg(reinterpret_cast<const float4 *>(row_parts + ((s0 + s + u) * G + h) * kPartialStride) + c4);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float wgt = wts[(s + u) * G + h];
+            acc.x += wgt * v[u].x;
+            acc.y += wgt * v[u].y;
+            acc.z += wgt * v[u].z;
+            acc.w += wgt * v[u].w;
+          }
+        }
+        for (; s < cnt; ++s) {
+          const float4 v = __ldcg(reinterpret_cast<const float4 *>(row_parts + ((s0 + s) * G + h) * kPartialStride) + c4);
+          const float wgt = wts[s * G + h];
+          acc.x += wgt * v.x;
+          acc.y += wgt * v.y;
+          acc.z += wgt * v.z;
+          acc.w += wgt * v.w;
+        }
+        if (half) o1 = acc; else o0 = acc;
+      }
+    }
+    named_barrier(1, kAttnThreads);
+  }
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int fi = f + half * kAttnThreads;
+    if (fi < G * 32) {
+      const float4 acc = half ? o1 : o0;
+      const uint32_t lo = pack_bf16x2(acc.x, acc.y), hi = pack_bf16x2(acc.z, acc.w);
+      *reinterpret_cast<uint2 *>(out_rows + (fi >> 5) * kHeadDim + 4 * (fi & 31)) = make_uint2(lo, hi);
+    }
+  }
+  // mask row: each word gathers 32 consecutive blocks' bits from the split
+  // bit rows, loading each split word once
   const uint32_t *row_bits = p.split_bits + row * p.nsplit_max * p.split_words;
   for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads) {
-    uint32_t bits = 0;
+    uint32_t bits = 0, cached = 0;
+    int key = -1;
     for (int k = 0; k < 32; ++k) {
       const int j = 32 * w + k;
-      if (j < nb) {
-        const int s = j / p.split_blocks, i = j - s * p.split_blocks;
-        bits |= ((__ldcg(row_bits + s * p.split_words + (i >> 5)) >> (i & 31)) & 1u) << k;
+      if (j >= nb) break;
+      const int s = j / p.split_blocks, i = j - s * p.split_blocks;
+      const int kk = s * p.split_words + (i >> 5);
+      if (kk != key) {
+        cached = __ldcg(row_bits + kk);
+        key = kk;
       }
+      bits |= ((cached >> (i & 31)) & 1u) << k;
     }
     p.mask[row * p.mask_words + w] = bits;
   }
