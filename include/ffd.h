@@ -143,6 +143,19 @@ ffd_status ffd_decode(const ffd_shape *shape, const void *q_bf16, const void *k_
                       const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                       void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* The whole decode step in one launch: re-quantise each sequence's last key
+ * block (exactly ffd_quantize_keys with FFD_LAST_BLOCK: the caller has just
+ * appended the current token's K/V at position lengths[b] - 1), then run
+ * ffd_decode.  The CTA that owns a sequence's last split does the
+ * re-quantisation before its scan, so no other work waits for it.
+ * k_packed and k_scales are read and (for the last block) written; they are
+ * required even when delta == +INFINITY.  Results are bit-identical to the
+ * two calls in sequence. */
+ffd_status ffd_decode_step(const ffd_shape *shape, const void *q_bf16, const void *k_bf16,
+                           const void *v_bf16, void *k_packed, void *k_scales,
+                           const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                           void *workspace, size_t workspace_bytes, void *cuda_stream);
+
 /* ffd_decode without a caller workspace, for callers that cannot allocate
  * device memory: e.g. a plug-in inside an inference engine that is given only
  * its input and output buffers, or a serving loop that must not call

@@ -178,10 +178,13 @@ ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32
   return FFD_OK;
 }
 
-ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16, const void *v_bf16,
-                      const void *k_packed, const void *k_scales, const int32_t *d_lengths, float delta,
-                      void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
-                      void *cuda_stream) {
+namespace {
+
+// Shared body of ffd_decode and ffd_decode_step.
+ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
+                         const void *v_bf16, const void *k_packed, const void *k_scales,
+                         const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                         void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (std::isnan(delta) || delta < 0.0f) return FFD_ERR_INVALID_ARG;
@@ -194,11 +197,12 @@ ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16
   if (q_bf16 == nullptr || k_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
       out_bf16 == nullptr || mask == nullptr)
     return FFD_ERR_INVALID_ARG;
-  if (!dense && (k_packed == nullptr || k_scales == nullptr)) return FFD_ERR_INVALID_ARG;
+  const bool need_packed = requant || !dense;
+  if (need_packed && (k_packed == nullptr || k_scales == nullptr)) return FFD_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
       !aligned16(mask) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
     return FFD_ERR_INVALID_ARG;
-  if (!dense && (!aligned16(k_packed) || !aligned16(k_scales))) return FFD_ERR_INVALID_ARG;
+  if (need_packed && (!aligned16(k_packed) || !aligned16(k_scales))) return FFD_ERR_INVALID_ARG;
 
   const uint64_t rows = static_cast<uint64_t>(s->batch) * s->num_kv_heads * s->capacity;
   CUtensorMap tmap_k, tmap_v;
@@ -226,6 +230,10 @@ ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16
   p.split_words = L.split_words;
   p.delta = delta;
   p.dense = dense ? 1 : 0;
+  p.requant_last = requant ? 1 : 0;
+  p.k = static_cast<const uint16_t *>(k_bf16);
+  p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(k_packed)) : nullptr;
+  p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(k_scales)) : nullptr;
 
   const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
                   static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
@@ -234,6 +242,24 @@ ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16
                     static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
     return FFD_ERR_CUDA;
   return FFD_OK;
+}
+
+}  // namespace
+
+ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                      const void *k_packed, const void *k_scales, const int32_t *d_lengths, float delta,
+                      void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
+                      void *cuda_stream) {
+  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+                       mask, workspace, workspace_bytes, cuda_stream, false);
+}
+
+ffd_status ffd_decode_step(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
+                           const void *v_bf16, void *k_packed, void *k_scales,
+                           const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                           void *workspace, size_t workspace_bytes, void *cuda_stream) {
+  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+                       mask, workspace, workspace_bytes, cuda_stream, true);
 }
 
 ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream) {

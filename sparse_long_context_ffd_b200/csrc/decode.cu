@@ -35,6 +35,7 @@
 #include "ffd.h"
 #include "ffd_internal.h"
 #include "ffd_ptx.cuh"
+#include "ffd_quant.cuh"
 
 namespace ffd {
 namespace {
@@ -279,6 +280,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
+  }
+  // Fused decode step: the CTA that owns a sequence's last block re-quantises
+  // it (the appended token changed it) before anything reads the int4 copy;
+  // the generic-proxy stores are fenced before the bulk copies read them.
+  if (p.requant_last && split == nsplit - 1) {
+    if (threadIdx.x < kAttnThreads) {
+      const int jl = nb - 1;
+      const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
+      float *red = reinterpret_cast<float *>(scan_ring);  // idle until the scan starts
+      quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                      p.packed_out + tok0 * kPackedRowBytes,
+                                      p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim,
+                                      red, red + (kAttnThreads / 32) * kHeadDim,
+                                      static_cast<int>(threadIdx.x), 2);
+      fence_proxy_async_global();
+    }
+    fence_proxy_async_smem();
   }
   __syncthreads();
 
@@ -635,44 +653,53 @@ __global__ void __launch_bounds__(kThreads, 2)
   __threadfence();
 
   // last CTA of (b, g): log-sum-exp merge over the splits.  Every load here
-  // is independent of the others, so the merge costs a few L2 round trips
-  // rather than one per split:
-  //   1. per head (one warp per head, lanes striding over the splits):
-  //      M* = max_s m_s and L* = sum_s l_s 2^(m_s - M*);
-  //   2. in chunks of splits: weights 2^(m_s - M*) / L* into shared memory,
-  //      then each thread accumulates four output channels with float4 loads.
+  // is independent of the others, so the merge costs about three L2 round
+  // trips rather than one per split:
+  //   1. per head (one warp per head, lanes striding over the splits): the
+  //      split maxima and sums are combined pairwise, (m1, l1) + (m2, l2) =
+  //      (M, l1 2^(m1 - M) + l2 2^(m2 - M)), into M* and L*; the split maxima
+  //      of the first chunk stay in shared memory;
+  //   2. per chunk of splits: weights 2^(m_s - M*) / L* in shared memory,
+  //      then each thread accumulates four output channels with float4 loads
+  //      issued sixteen at a time.
   const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
   float *stats = reinterpret_cast<float *>(scan_ring);  // [G][2]: M*, L*
   float *wts = stats + 16;                              // [chunk][G]
+  constexpr int kWtsFloats = ScanGeom<T>::kRingBytes / 4 - 16;
+  const int chunk = kWtsFloats / G;
   for (int h = warp; h < G; h += kAttnWarps) {
-    float m = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32)
-      m = fmaxf(m, __ldcg(row_parts + (s * G + h) * kPartialStride + 128));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
-    float l = 0.0f;
+    float m = -INFINITY, l = 0.0f;
     for (int s = lane; s < nsplit; s += 32) {
       const float *ps = row_parts + (s * G + h) * kPartialStride;
-      l += __ldcg(ps + 129) * exp2f(__ldcg(ps + 128) - m);
+      const float ms = __ldcg(ps + 128), ls = __ldcg(ps + 129);
+      if (s < chunk) wts[s * G + h] = ms;
+      const float mn = fmaxf(m, ms);  // ms is finite: every split keeps a valid token
+      l = l * exp2f(m - mn) + ls * exp2f(ms - mn);
+      m = mn;
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFull, l, off);
+    for (int off = 16; off > 0; off >>= 1) {
+      const float mo = __shfl_xor_sync(kFull, m, off), lo = __shfl_xor_sync(kFull, l, off);
+      const float mn = fmaxf(m, mo);
+      if (mn != -INFINITY) {
+        l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mn));
+        m = mn;
+      }
+    }
     if (lane == 0) {
       stats[2 * h] = m;
       stats[2 * h + 1] = l;
     }
   }
   named_barrier(1, kAttnThreads);
-  constexpr int kWtsFloats = ScanGeom<T>::kRingBytes / 4 - 16;
-  const int chunk = kWtsFloats / G;
   const int f = threadIdx.x;  // float4 output index: head f / 32, channels 4 (f % 32) ..
   float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;  // second set for G == 8
   for (int s0 = 0; s0 < nsplit; s0 += chunk) {
     const int cnt = min(chunk, nsplit - s0);
     for (int i = threadIdx.x; i < cnt * G; i += kAttnThreads) {
       const int h = i % G, s = s0 + i / G;
-      wts[i] = exp2f(__ldcg(row_parts + (s * G + h) * kPartialStride + 128) - stats[2 * h]) /
-               stats[2 * h + 1];
+      const float ms = s0 == 0 ? wts[i] : __ldcg(row_parts + (s * G + h) * kPartialStride + 128);
+      wts[i] = exp2f(ms - stats[2 * h]) / stats[2 * h + 1];
     }
     named_barrier(1, kAttnThreads);
 #pragma unroll
@@ -682,13 +709,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int h = fi >> 5, c4 = fi & 31;
         float4 acc = half ? o1 : o0;
         int s = 0;
-        for (; s + 8 <= cnt; s += 8) {
-          float4 v[8];
+        for (; s + 16 <= cnt; s += 16) {
+          float4 v[16];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
+          for (int u = 0; u < 16; ++u)
             v[u] = __ldcg(reinterpret_cast<const float4 *>(row_parts + ((s0 + s + u) * G + h) * kPartialStride) + c4);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int u = 0; u < 16; ++u) {
             const float wgt = wts[(s + u) * G + h];
             acc.x += wgt * v[u].x;
             acc.y += wgt * v[u].y;

@@ -37,6 +37,11 @@ struct DecodeParams {
   int32_t batch, num_kv_heads, capacity, split_blocks, nsplit_max, mask_words, split_words;
   float delta;
   int32_t dense;
+  // fused decode step: re-quantise each sequence's last key block first
+  int32_t requant_last;
+  const uint16_t *k;         // bf16 [B][Hkv][cap][D] (read by the re-quantisation)
+  uint8_t *packed_out;       // = packed, written for the last block
+  uint16_t *scales_out;      // = scales, written for the last block
 };
 
 struct QuantizeParams {

@@ -1,0 +1,100 @@
+// ffd_quant.cuh -- quantisation of one key block to the int4 scan copy,
+// shared by the quantize kernel and the fused decode step.
+//
+// The low-bit key "thumbnail" (Faster Than Flash, gist.science explainer,
+// Methodology 1): symmetric int4 codes in [-7, 7] with one bf16 scale per
+// (block, channel), scale = bf16_rne(amax / 7) by IEEE division, code =
+// clamp(rint_even(k / scale), -7, 7), nibble = code + 8, byte i of a token row
+// = channel 2i (low nibble) | channel 2i+1 (high nibble).  Tokens at or past
+// the sequence length are excluded from amax and stored as code 0.  Every
+// step is one correctly rounded IEEE operation, so the result is bit-exact.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "ffd_internal.h"
+#include "ffd_ptx.cuh"
+
+namespace ffd {
+
+__device__ __forceinline__ float q_bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float q_bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// NT threads (a multiple of 32, at least 32, tid in [0, NT)) quantise one
+// block of T token rows.  Thread (rg = tid / 16, cg = tid % 16) owns channels
+// 8cg .. 8cg+7 of rows rg, rg + NT/16, ...: one 16-byte load and one 4-byte
+// store of 8 nibbles per row.  red holds NT/32 x 128 floats and scale_s 128
+// floats of shared memory; `bar_id` names a barrier used by exactly these NT
+// threads.
+template <int T, int NT>
+__device__ __forceinline__ void quantize_block(const uint16_t *k_rows, int valid, uint8_t *packed_rows,
+                                               uint16_t *scale_row, float *red, float *scale_s, int tid,
+                                               uint32_t bar_id) {
+  static_assert(NT % 32 == 0 && NT >= 32 && T % (NT / 16) == 0, "thread layout");
+  constexpr int RG = NT / 16;  // row groups
+  constexpr int R = T / RG;    // rows per thread
+  const int cg = tid & 15;
+  const int rg = tid >> 4;
+  uint4 x[R];
+  float amax[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) amax[c] = 0.0f;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int t = rg + RG * r;
+    if (t < valid) {
+      x[r] = *reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 8 * cg);
+      const uint32_t w[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        amax[2 * e] = fmaxf(amax[2 * e], fabsf(q_bf16_lo(w[e])));
+        amax[2 * e + 1] = fmaxf(amax[2 * e + 1], fabsf(q_bf16_hi(w[e])));
+      }
+    } else {
+      x[r] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  // row groups rg and rg ^ 1 share a warp and differ in bit 4 of the lane id
+#pragma unroll
+  for (int c = 0; c < 8; ++c) amax[c] = fmaxf(amax[c], __shfl_xor_sync(0xFFFFFFFFu, amax[c], 16));
+  const int warp = tid >> 5;
+  if ((tid & 16) == 0) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) red[warp * kHeadDim + 8 * cg + c] = amax[c];
+  }
+  named_barrier(bar_id, NT);
+  if (tid < kHeadDim) {
+    float a = red[tid];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) a = fmaxf(a, red[w * kHeadDim + tid]);
+    const __nv_bfloat16 s = __float2bfloat16_rn(__fdiv_rn(a, 7.0f));
+    scale_row[tid] = __bfloat16_as_ushort(s);
+    scale_s[tid] = __bfloat162float(s);
+  }
+  named_barrier(bar_id, NT);
+  float sf[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) sf[c] = scale_s[8 * cg + c];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int t = rg + RG * r;
+    const uint32_t w[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
+    uint32_t nibbles = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float v = (c & 1) ? q_bf16_hi(w[c >> 1]) : q_bf16_lo(w[c >> 1]);
+      int code = 0;
+      if (t < valid && sf[c] != 0.0f) {
+        code = __float2int_rn(__fdiv_rn(v, sf[c]));
+        code = min(7, max(-7, code));
+      }
+      nibbles |= static_cast<uint32_t>(code + 8) << (4 * c);
+    }
+    *reinterpret_cast<uint32_t *>(packed_rows + static_cast<size_t>(t) * kPackedRowBytes + 4 * cg) =
+        nibbles;
+  }
+}
+
+}  // namespace ffd

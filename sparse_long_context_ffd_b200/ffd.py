@@ -32,7 +32,7 @@ FFD_MAX_SPLIT_BLOCKS = 512
 EXPORTED = (
     "ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words", "ffd_decode_workspace_bytes",
     "ffd_workspace_init", "ffd_quantize_keys", "ffd_decode", "ffd_check_device_status",
-    "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc",
+    "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc", "ffd_decode_step",
 )
 
 # Size of the library's built-in scratch array used by ffd_decode_no_alloc.
@@ -88,6 +88,8 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_quantize_keys.restype = st
             lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode.restype = st
+            lib.ffd_decode_step.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
+            lib.ffd_decode_step.restype = st
             lib.ffd_decode_no_alloc.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p]
             lib.ffd_decode_no_alloc.restype = st
             lib.ffd_check_device_status.argtypes = [p, ctypes.POINTER(ctypes.c_uint32), p]
@@ -169,6 +171,16 @@ def decode(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out
                                       float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "ffd_decode")
+
+
+def decode_step(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out, mask,
+                workspace, stream=None) -> None:
+    """Re-quantise each sequence's last key block and decode, in one launch."""
+    _check(load_library().ffd_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
+                                           float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)), "ffd_decode_step")
 
 
 def decode_no_alloc(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out,

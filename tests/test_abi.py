@@ -113,6 +113,11 @@ def test_bad_arguments_rejected_on_host():
                           a, 1 << 20, None) == ffd.FFD_OK
     assert lib.ffd_workspace_init(ctypes.byref(s), a, ws - 1, None) == ffd.FFD_ERR_WORKSPACE
     assert lib.ffd_check_device_status(None, None, None) == ffd.FFD_ERR_INVALID_ARG
+    # the fused step writes the int4 copy, so it needs it even in dense mode
+    assert lib.ffd_decode_step(ctypes.byref(s), a, a, a, None, a, a, float("inf"), a, a, a, ws,
+                               None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_decode_step(ctypes.byref(s), a, a, a, a, a, a, -1.0, a, a, a, ws,
+                               None) == ffd.FFD_ERR_INVALID_ARG
 
 
 def test_product_path_never_touches_the_oracle():

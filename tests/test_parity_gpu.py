@@ -240,3 +240,37 @@ def test_full_config(name):
 def test_max256k_delta_sweep():
     rep = _full_config("max256k", list(fw.MAX256K_DELTAS))
     print("max256k", rep)
+
+
+# ------------------------------------------------- fused step (append path) --
+
+@pytest.mark.parametrize("T,delta", [(64, 2.0), (128, 0.75), (64, INF)])
+def test_decode_step_equals_quantize_then_decode(T, delta):
+    # inputs drawn for the final lengths; decoding starts 5 tokens earlier and
+    # appends one token per step (the data past the current length is real)
+    w = fw.random_small_workload(50 + T, 3, 4, 2, 32 * T, T, 5, 2.0, 6 * T, 32 * T, needles=2)
+    inp = fw.make_inputs(w)
+    final = inp["lengths"].copy()
+    a = GpuCase(w, inp, lengths=final - 5)
+    b = GpuCase(w, inp, lengths=final - 5)
+    a.quantize(0)
+    b.quantize(0)
+    for step in range(5):
+        ln = torch.from_numpy(final - 4 + step).cuda()
+        a.lengths.copy_(ln)
+        b.lengths.copy_(ln)
+        ffd.decode_step(a.shape, a.q, a.k, a.v, a.bufs.k_packed, a.bufs.k_scales, a.lengths, delta,
+                        a.bufs.out, a.bufs.mask, a.bufs.workspace)
+        b.quantize(ffd.FFD_LAST_BLOCK)
+        ffd.decode(b.shape, b.q, b.k, b.v, b.bufs.k_packed, b.bufs.k_scales, b.lengths, delta,
+                   b.bufs.out, b.bufs.mask, b.bufs.workspace)
+        torch.cuda.synchronize()
+        assert torch.equal(a.bufs.out.view(torch.int16), b.bufs.out.view(torch.int16))
+        assert torch.equal(a.bufs.mask, b.bufs.mask)
+        assert torch.equal(a.bufs.k_packed, b.bufs.k_packed)
+        assert torch.equal(a.bufs.k_scales.view(torch.int16), b.bufs.k_scales.view(torch.int16))
+    want_out, want_mask, _, _ = _oracle(w, inp, delta, lengths=final)
+    from gpu_util import bf16_to_np_f32
+    assert_mask_equal(a.bufs.mask.cpu().numpy().view(np.uint32), want_mask, f"step T{T} {delta}")
+    assert_output_close(bf16_to_np_f32(a.bufs.out).astype(np.float64), want_out, f"step T{T} {delta}")
+    assert ffd.check_device_status(a.bufs.workspace) == 0
