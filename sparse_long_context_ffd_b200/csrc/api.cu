@@ -53,17 +53,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// K or V cache viewed as rows of 128 bf16 (256 bytes); boxes of 64 channels
-// x kKvBoxRows tokens with the 128-byte swizzle (one box = one 64-channel
-// half of an attention pipeline stage).
+// K or V cache as a 3-D tensor {64 channels, token rows, 2 halves}: a row is
+// 128 bf16 (256 bytes) and a half its low or high 128 bytes.  One box
+// {64, kKvBoxRows, 2} is one attention stage's K (or V) tile; the 128-byte
+// swizzle applies per 128-byte box row, and shared memory receives the tile
+// as [half][row][64 channels].
 bool make_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), rows > 0 ? rows : 1};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kKvBoxRows)};
-  const cuuint32_t elem_strides[2] = {1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+  const cuuint64_t dims[3] = {64, rows > 0 ? rows : 1, 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kKvBoxRows), 2};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                             strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -15,7 +15,7 @@
 //   producer warp (one lane): an event loop that streams the split's packed
 //     key tiles and scales into the scan ring with 1-D bulk copies and, as
 //     kept blocks appear in the selection queue, their K and V into the
-//     attention ring with 2-D TMA copies (128-byte swizzle);
+//     attention ring with one 3-D TMA copy each (128-byte swizzle);
 //   scan warp: folds the query group into int8 for each block, scores all
 //     tokens on the tensor cores (mma m16n8k32, u8 nibbles x s8 query), keeps
 //     the per-head running maximum in registers, applies the Top-delta test,
@@ -349,10 +349,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         seq[st] = it_next;
         mbar_arrive_expect_tx(&full_b[st], kKvStageBytes);
         const int y = row_tok0 + tok;
-        tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);
-        tma_load_2d(dst + kKvHalfBytes, &tmap_k, 64, y, &full_b[st]);
-        tma_load_2d(dst + 2 * kKvHalfBytes, &tmap_v, 0, y, &full_b[st]);
-        tma_load_2d(dst + 3 * kKvHalfBytes, &tmap_v, 64, y, &full_b[st]);
+        tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);                 // K: both halves
+        tma_load_3d(dst + 2 * kKvHalfBytes, &tmap_v, 0, y, 0, &full_b[st]);  // V: both halves
         ++it_next;
         ++sub;
         progress = true;

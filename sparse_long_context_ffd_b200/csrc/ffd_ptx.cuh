@@ -107,6 +107,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int32_t
       : "memory");
 }
 
+// 3-D tiled tensor copy global -> shared through a CUtensorMap (TMA).
+__device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, int32_t x, int32_t y,
+                                            int32_t z, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
