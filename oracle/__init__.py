@@ -55,6 +55,8 @@ def _load():
             lib.ffdo_attend.argtypes = [i, i, i, i, i, i, p, p, p, p, p, p, p]
             lib.ffdo_decode.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p,
                                         ctypes.c_float, p, p, p]
+            lib.ffdo_decode_pseudo_max.argtypes = lib.ffdo_decode.argtypes
+            lib.ffdo_select_pseudo_max.argtypes = lib.ffdo_select.argtypes
             _lib = lib
     return _lib
 
@@ -113,15 +115,19 @@ def block_scores(q, packed, scales, lengths, block_size):
     return out
 
 
-def select(scores, lengths, num_kv_heads, capacity, block_size, split_blocks, delta):
-    """Returns (keep [B,Hq,nblk] uint8, mask [B,Hkv,words] uint32)."""
+def select(scores, lengths, num_kv_heads, capacity, block_size, split_blocks, delta,
+           pseudo_max=False):
+    """Returns (keep [B,Hq,nblk] uint8, mask [B,Hkv,words] uint32).  pseudo_max
+    selects the sink/local reference maximum instead of starting each split's
+    running maximum at minus infinity."""
     scores = _c(scores, np.float32)
     lengths = _c(lengths, np.int32)
     B, Hq, nblk = scores.shape
     keep = np.zeros((B, Hq, nblk), dtype=np.uint8)
     mask = np.zeros((B, num_kv_heads, mask_words(capacity, block_size)), dtype=np.uint32)
-    _check(_load().ffdo_select(B, Hq, num_kv_heads, capacity, block_size, split_blocks,
-                               _ptr(scores), _ptr(lengths), float(delta), _ptr(keep), _ptr(mask)))
+    fn = _load().ffdo_select_pseudo_max if pseudo_max else _load().ffdo_select
+    _check(fn(B, Hq, num_kv_heads, capacity, block_size, split_blocks, _ptr(scores), _ptr(lengths),
+              float(delta), _ptr(keep), _ptr(mask)))
     return keep, mask
 
 
@@ -141,7 +147,7 @@ def attend(q, k, v, lengths, mask, block_size):
     return out, lse
 
 
-def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta):
+def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta, pseudo_max=False):
     """The whole step.  Returns (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores)."""
     q = _c(q, np.uint16)
     k = _c(k, np.uint16)
@@ -154,9 +160,10 @@ def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta):
     out = np.zeros((B, Hq, D), dtype=np.float64)
     mask = np.zeros((B, Hkv, mask_words(cap, block_size)), dtype=np.uint32)
     scores = np.zeros((B, Hq, cap // block_size), dtype=np.float32)
-    _check(_load().ffdo_decode(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(k),
-                               _ptr(v), _ptr(packed), _ptr(scales), _ptr(lengths), float(delta),
-                               _ptr(out), _ptr(mask), _ptr(scores)))
+    fn = _load().ffdo_decode_pseudo_max if pseudo_max else _load().ffdo_decode
+    _check(fn(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(k), _ptr(v),
+              _ptr(packed), _ptr(scales), _ptr(lengths), float(delta), _ptr(out), _ptr(mask),
+              _ptr(scores)))
     return out, mask, scores
 
 

@@ -29,6 +29,9 @@
  *   R7  the query is the last token: no causal mask; tokens >= length never
  *       contribute.
  *   R13 a sequence of length 0 yields a zero output row and an empty mask.
+ *   R15 pseudo-max reference (optional mode): the sink tokens are block 0,
+ *       the local tokens the last block; the split's running maximum starts
+ *       at the larger of their two block scores.
  *
  * Floating point: the selection steps use fp32 with one IEEE operation per
  * step (this file must be built with -ffp-contract=off and without fast-math);
@@ -253,6 +256,47 @@ int ffdo_select(int B, int Hq, int Hkv, int cap, int T, int S, const float *scor
   return FFDO_OK;
 }
 
+/* ---- step 4': Top-delta with the pseudo-max reference (gist.science,
+ *      Methodology 2, "Pseudo-Max Approximation": the reference maximum is
+ *      estimated from the sink tokens and the local tokens only; R15) -------
+ * Per head h the pseudo-max is mt_h = max(s_{0,h}, s_{nb-1,h}) (the first and
+ * the last block of the sequence).  Inside each split, in ascending order,
+ * m = max(m, s_j) starting from m = mt_h, and block j is kept for h iff
+ * s_j >= m - delta.  Splits stay independent; a split may keep nothing. */
+int ffdo_select_pseudo_max(int B, int Hq, int Hkv, int cap, int T, int S, const float *scores,
+                           const int32_t *lengths, float delta, uint8_t *keep, uint32_t *mask) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || T <= 0 || cap % T != 0 || S <= 0)
+    return FFDO_BAD_ARG;
+  if (!(delta >= 0.0f)) return FFDO_BAD_ARG;
+  int G = Hq / Hkv, nblk = cap / T, words = (nblk + 31) / 32;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 0 || lengths[b] > cap) return FFDO_BAD_LENGTH;
+  memset(mask, 0, sizeof(uint32_t) * (size_t)B * Hkv * words);
+  if (keep) memset(keep, 0, (size_t)B * Hq * nblk);
+  for (int b = 0; b < B; ++b) {
+    int nb = (lengths[b] + T - 1) / T;
+    if (nb == 0) continue;
+    for (int h = 0; h < Hq; ++h) {
+      int g = h / G;
+      const float *s = scores + ((size_t)b * Hq + h) * nblk;
+      uint32_t *m = mask + ((size_t)b * Hkv + g) * words;
+      float pseudo = fmaxf(s[0], s[nb - 1]);
+      for (int split0 = 0; split0 < nb; split0 += S) {
+        int split1 = split0 + S < nb ? split0 + S : nb;
+        float running = pseudo;
+        for (int j = split0; j < split1; ++j) {
+          running = fmaxf(running, s[j]);
+          float threshold = running - delta;
+          int k = s[j] >= threshold;
+          if (keep) keep[((size_t)b * Hq + h) * nblk + j] = (uint8_t)k;
+          if (k) m[j / 32] |= 1u << (j % 32);
+        }
+      }
+    }
+  }
+  return FFDO_OK;
+}
+
 /* ---- step 5: exact attention over the selected blocks (gist.science,
  *      Methodology 3, stage "Fine-Grained Refinement"; R6, R7), fp64 -------- */
 
@@ -315,10 +359,32 @@ int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
 
 /* delta = +INF selects every valid block (dense attention).  scores may be NULL
  * (a scratch buffer is allocated); packed/scales may be NULL when delta = +INF. */
+static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
+                       const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
+                       float delta, double *out, uint32_t *mask, float *scores, int pseudo_max);
+
 int ffdo_decode(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                 const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
                 float delta, double *out, uint32_t *mask, float *scores) {
+  return decode_impl(B, Hq, Hkv, cap, D, T, S, q, k, v, packed, scales, lengths, delta, out,
+                     mask, scores, 0);
+}
+
+/* The whole step with the pseudo-max reference (R15). */
+int ffdo_decode_pseudo_max(int B, int Hq, int Hkv, int cap, int D, int T, int S,
+                           const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
+                           float delta, double *out, uint32_t *mask, float *scores) {
+  return decode_impl(B, Hq, Hkv, cap, D, T, S, q, k, v, packed, scales, lengths, delta, out,
+                     mask, scores, 1);
+}
+
+static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
+                       const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
+                       float delta, double *out, uint32_t *mask, float *scores, int pseudo_max) {
   int rc = check_shape(B, Hq, Hkv, cap, D, T);
   if (rc != FFDO_OK) return rc;
   if (S <= 0 || !(delta >= 0.0f)) return FFDO_BAD_ARG;
@@ -337,7 +403,9 @@ int ffdo_decode(int B, int Hq, int Hkv, int cap, int D, int T, int S,
     rc = ffdo_block_scores(B, Hq, Hkv, cap, D, T, q, packed, scales, lengths, scores);
     if (rc != FFDO_OK) { free(own); return rc; }
   }
-  rc = ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  rc = pseudo_max
+           ? ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask)
+           : ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
   if (rc == FFDO_OK) rc = ffdo_attend(B, Hq, Hkv, cap, D, T, q, k, v, lengths, mask, out, NULL);
   free(own);
   return rc;

@@ -552,3 +552,101 @@ def test_planted_needles_are_selected(name, overrides):
                     assert bits[j], (name, delta, b, g, j)
                     # the targeted head keeps it on its own
                     assert keep[b, g * w.group + i % w.group, j]
+
+
+# ------------------------------------------- pseudo-max reference (sink/local) --
+
+def test_select_pseudo_max_hand_worked_example():
+    meta, cases = {}, []
+    with open(os.path.join(GOLDEN, "topdelta_pseudo_max_example.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            if key == "case":
+                cases.append(dict(item.split("=") for item in rest))
+            else:
+                meta[key] = rest
+    T, S, nb = int(meta["block_size"][0]), int(meta["split_blocks"][0]), int(meta["num_blocks"][0])
+    scores = np.array([[list(map(float, meta["scores_head0"]))]], np.float32)
+    lengths = np.array([nb * T], np.int32)
+    assert len(cases) == 4
+    for case in cases:
+        _, mask = oracle.select(scores, lengths, 1, nb * T, T, S, float(case["delta"]),
+                                pseudo_max=case["reference"] == "pseudo")
+        assert int(mask[0, 0, 0]) == int(case["mask"], 16), case
+
+
+def _declarative_keep_pseudo(s, nb, S, delta):
+    """keep_j <=> s_j >= max(pseudo, s over j's split up to j) - delta, with
+    pseudo = max(s_0, s_{nb-1})."""
+    pseudo = max(s[0], s[nb - 1])
+    out = np.zeros(nb, bool)
+    for j in range(nb):
+        start = (j // S) * S
+        ref = max(pseudo, max(s[start:j + 1]))
+        out[j] = s[j] >= np.float32(np.float32(ref) - np.float32(delta))
+    return out
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_pseudo_max_matches_bruteforce_enumeration(seed):
+    rng = np.random.default_rng(300 + seed)
+    for _ in range(8):
+        nb = int(rng.integers(1, 13))
+        S = int(rng.choice([1, 3, 4, nb]))
+        G = int(rng.choice([1, 4]))
+        T = 64
+        scores = (rng.integers(-8, 9, size=(1, G, nb)) * 0.5).astype(np.float32)
+        delta = float(rng.choice([0.0, 0.5, 1.0, 2.5, np.inf]))
+        _, mask = oracle.select(scores, np.array([nb * T], np.int32), 1, nb * T, T, S, delta,
+                                pseudo_max=True)
+        got = oracle.mask_to_blocks(mask[0, 0], nb)
+        per_head = [_declarative_keep_pseudo(scores[0, h], nb, S, delta) for h in range(G)]
+        satisfying = [np.array(bits) for bits in itertools.product([False, True], repeat=nb)
+                      if all(bits[j] == any(ph[j] for ph in per_head) for j in range(nb))]
+        assert len(satisfying) == 1 and np.array_equal(satisfying[0], got)
+
+
+def test_select_pseudo_max_invariants():
+    rng = np.random.default_rng(31)
+    B, G, Hkv, T, S, nblk = 2, 4, 2, 64, 5, 23
+    lengths = np.array([nblk * T, 9 * T + 3], np.int32)
+    scores = rng.standard_normal((B, G * Hkv, nblk)).astype(np.float32)
+    for b in range(B):
+        scores[b, :, -(-int(lengths[b]) // T):] = -np.inf
+    cap = nblk * T
+    prev = None
+    for d in [0.0, 0.25, 0.5, 1.0, 2.0, 4.0, np.inf]:
+        keep_p, mask_p = oracle.select(scores, lengths, Hkv, cap, T, S, d, pseudo_max=True)
+        _, mask_r = oracle.select(scores, lengths, Hkv, cap, T, S, d)
+        cur = np.array([[oracle.mask_to_blocks(mask_p[b, g], nblk) for g in range(Hkv)]
+                        for b in range(B)])
+        run = np.array([[oracle.mask_to_blocks(mask_r[b, g], nblk) for g in range(Hkv)]
+                        for b in range(B)])
+        assert (cur <= run).all()  # a higher reference keeps a subset
+        if prev is not None:
+            assert (prev <= cur).all()  # monotone in delta
+        prev = cur
+        for b in range(B):
+            nb = -(-int(lengths[b]) // T)
+            for h in range(G * Hkv):
+                # the head's highest-scoring block is always kept (no head keeps nothing)
+                assert keep_p[b, h, int(np.argmax(scores[b, h, :nb]))]
+                # block 0 opens its split, so it is kept whenever it sets the pseudo-max
+                if scores[b, h, 0] >= scores[b, h, nb - 1]:
+                    assert keep_p[b, h, 0]
+            if d == np.inf:
+                assert cur[b, :, :nb].all()
+
+
+def test_decode_pseudo_max_attends_over_its_mask():
+    w, inp = _rand_case(77, B=3, G=4, Hkv=2, cap=2048, T=64, S=4, lo=300, hi=2048)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    for delta in (0.0, 1.0):
+        out, mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales, inp["lengths"],
+                                     w.block_size, w.split_blocks, delta, pseudo_max=True)
+        ref = _library_attention(inp["q"], inp["k"], inp["v"], inp["lengths"],
+                                 _token_keep(mask, w.block_size, w.capacity))
+        np.testing.assert_allclose(out, ref, atol=1e-10)
