@@ -42,6 +42,7 @@ if ROOT not in sys.path:
 import ffd_workloads as fw  # noqa: E402
 
 DEFAULT_WORKLOAD = "long128k"
+REFERENCES = {"running": 0, "sink_local": 1}  # FFD_REFERENCE_* of include/ffd.h
 METRIC = "us per decode step (128K ctx) + effective HBM TB/s of the fused decode kernel"
 UNIT = "us/step"
 
@@ -274,6 +275,8 @@ class Replica:
             self.layers.append(layer)
         torch.cuda.synchronize(device)
 
+    reference = 0  # FFD_REFERENCE_RUNNING_MAX; set from --reference
+
     def step(self, i, delta, ev=None, fused=True):
         """One decode step: re-quantise the last key block, then the fused
         decode -- one launch (ffd_decode_step), or two (ffd_quantize_keys +
@@ -285,9 +288,9 @@ class Replica:
                                    b.k_packed, b.k_scales)
         if ev is not None:
             ev[0].record()
-        call = self.ffd.decode_step if fused else self.ffd.decode
-        call(self.shape, L["q"], L["k"], L["v"], b.k_packed, b.k_scales, self.lengths, delta,
-             b.out, b.mask, b.workspace)
+        self.ffd.decode_ex(self.shape, L["q"], L["k"], L["v"], b.k_packed, b.k_scales,
+                           self.lengths, delta, b.out, b.mask, b.workspace,
+                           reference=self.reference, requant_last=fused)
         if ev is not None:
             ev[1].record()
 
@@ -521,6 +524,7 @@ def run_profile(args):
     delta = w.delta if args.delta is None else args.delta
     inp = fw.make_inputs(w)
     rep = Replica(w, inp, device, 1)
+    rep.reference = REFERENCES[args.reference]
     for i in range(args.profile_steps):
         rep.step(i, delta)
     torch.cuda.synchronize(device)
@@ -550,6 +554,7 @@ def run_gpu(args):
 
     # first pass: learn the kept set (same content on every layer copy)
     probe = Replica(w, inp, device, 1)
+    probe.reference = REFERENCES[args.reference]
     probe.step(0, w.delta)
     torch.cuda.synchronize(device)
     mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
@@ -560,6 +565,7 @@ def run_gpu(args):
     layers = max(1, min(64, math.ceil(3 * l2 / min(algo["total"], algo_dense["total"]))))
     del probe
     rep = Replica(w, inp, device, layers)
+    rep.reference = REFERENCES[args.reference]
 
     sampler = ClockSampler(device.index, os.path.join(ROOT, "gpurun_out", "clocks.csv")
                            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
@@ -614,6 +620,7 @@ def run_gpu(args):
             "dtype": "bf16 K/V + int4xint8 scan, fp32 accumulate",
             "data": "synthetic (seeded generator; stands in for RULER/LongBench inputs)",
             "config": {"workload": w.description, "name": w.name, "delta": w.delta,
+                       "reference": args.reference,
                        "kept_blocks": kept_blocks, "valid_blocks": valid_blocks,
                        "kept_fraction": kept_blocks / max(1, valid_blocks),
                        "l2": f"inputs rotated over {layers} cache copies "
@@ -658,6 +665,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ffd", "reference"], default="ffd")
     ap.add_argument("--workload", choices=sorted(fw.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--delta", type=float, default=None)
+    ap.add_argument("--reference", choices=sorted(REFERENCES), default="running",
+                    help="Top-delta reference maximum: running max in the split, or the "
+                         "pseudo-max of the sink and local blocks")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -156,6 +156,32 @@ ffd_status ffd_decode_step(const ffd_shape *shape, const void *q_bf16, const voi
                            const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                            void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* Reference maximum of the Top-delta filter. */
+#define FFD_REFERENCE_RUNNING_MAX 0 /* running max inside each split (default) */
+#define FFD_REFERENCE_SINK_LOCAL 1  /* pseudo-max from the sink and local blocks */
+
+typedef struct {
+  /* FFD_REFERENCE_RUNNING_MAX: each split's running maximum starts at -inf
+   *   (the first block of every split is kept).
+   * FFD_REFERENCE_SINK_LOCAL: the pseudo-max of gist.science explainer,
+   *   Methodology 2 "Pseudo-Max Approximation" -- the reference maximum is
+   *   estimated from the sink tokens and the local tokens only.  Here: per
+   *   query head, mt = max(score of block 0, score of block nb - 1), and each
+   *   split's running maximum starts at mt.  Every split still decides on its
+   *   own (each CTA scores those two blocks itself); a split may keep nothing;
+   *   the head's highest-scoring block is always kept. */
+  int32_t reference;
+  /* 1: re-quantise each sequence's last block first, as ffd_decode_step. */
+  int32_t requant_last;
+} ffd_decode_options;
+
+/* ffd_decode / ffd_decode_step with options (NULL is rejected).  k_packed
+ * and k_scales are written only when requant_last == 1. */
+ffd_status ffd_decode_ex(const ffd_shape *shape, const ffd_decode_options *options,
+                         const void *q_bf16, const void *k_bf16, const void *v_bf16, void *k_packed,
+                         void *k_scales, const int32_t *d_lengths, float delta, void *out_bf16,
+                         uint32_t *mask, void *workspace, size_t workspace_bytes, void *cuda_stream);
+
 /* ffd_decode without a caller workspace, for callers that cannot allocate
  * device memory: e.g. a plug-in inside an inference engine that is given only
  * its input and output buffers, or a serving loop that must not call

@@ -186,9 +186,12 @@ namespace {
 ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
                          const void *v_bf16, const void *k_packed, const void *k_scales,
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
-                         void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant) {
+                         void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
+                         int32_t reference) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
+  if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL)
+    return FFD_ERR_INVALID_ARG;
   if (std::isnan(delta) || delta < 0.0f) return FFD_ERR_INVALID_ARG;
   if (s->batch == 0) return FFD_OK;
   const bool dense = std::isinf(delta);
@@ -233,6 +236,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
   p.delta = delta;
   p.dense = dense ? 1 : 0;
   p.requant_last = requant ? 1 : 0;
+  p.reference = reference;
   p.k = static_cast<const uint16_t *>(k_bf16);
   p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(k_packed)) : nullptr;
   p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(k_scales)) : nullptr;
@@ -253,7 +257,7 @@ ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16
                       void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
                       void *cuda_stream) {
   return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
-                       mask, workspace, workspace_bytes, cuda_stream, false);
+                       mask, workspace, workspace_bytes, cuda_stream, false, FFD_REFERENCE_RUNNING_MAX);
 }
 
 ffd_status ffd_decode_step(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
@@ -261,7 +265,18 @@ ffd_status ffd_decode_step(const ffd_shape *s, const void *q_bf16, const void *k
                            const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                            void *workspace, size_t workspace_bytes, void *cuda_stream) {
   return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
-                       mask, workspace, workspace_bytes, cuda_stream, true);
+                       mask, workspace, workspace_bytes, cuda_stream, true, FFD_REFERENCE_RUNNING_MAX);
+}
+
+ffd_status ffd_decode_ex(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,
+                         const void *k_bf16, const void *v_bf16, void *k_packed, void *k_scales,
+                         const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                         void *workspace, size_t workspace_bytes, void *cuda_stream) {
+  if (opt == nullptr) return FFD_ERR_INVALID_ARG;
+  if (opt->requant_last != 0 && opt->requant_last != 1) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+                       mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
+                       opt->reference);
 }
 
 ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream) {

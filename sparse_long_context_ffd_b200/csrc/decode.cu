@@ -110,6 +110,12 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, int stages, int issue
     mbar_wait(&full[u % stages], static_cast<uint32_t>(u / stages) & 1u, kWaitLimitNs);
 }
 
+// Block index of scan entry e: with nref reference entries first (the sink
+// block 0, then the local block nb - 1), then the split's blocks from j0.
+__device__ __forceinline__ int scan_block_index(int e, int nref, int nb, int j0) {
+  return e < nref ? (e == 0 ? 0 : nb - 1) : j0 + (e - nref);
+}
+
 // Selector for one block (executed by one warp): fold the group's query with
 // the block's channel scales into int8, integer-score every token on the
 // tensor cores and return, in lane (0, t4), the scores of heads 2*t4 and
@@ -259,6 +265,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int j0 = split * p.split_blocks;
   const int nbs = min(p.split_blocks, nb - j0);
   const bool dense = p.dense != 0;
+  // pseudo-max reference: the scan first scores the sink block (0) and the
+  // local block (nb - 1), then the split's own blocks
+  const bool pseudo = p.reference != 0 && !dense;
+  const int nref = pseudo ? (nb > 1 ? 2 : 1) : 0;
+  // in the fused step the last block is being re-quantised by the CTA that
+  // owns it; every other CTA builds that block's int4 tile itself from K
+  const bool local_in_smem = pseudo && p.requant_last && nb > 1 && split != nsplit - 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSA; ++s) {
@@ -303,11 +316,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ================================================================ producer
   if (warp == kProducerWarp) {
     if (lane != 0) return;
-    const uint8_t *src_p =
-        p.packed + (row * p.capacity + static_cast<size_t>(j0) * T) * kPackedRowBytes;
-    const uint16_t *src_s = p.scales + (row * static_cast<size_t>(p.capacity / T) + j0) * kHeadDim;
+    const uint8_t *src_p = p.packed + row * p.capacity * kPackedRowBytes;
+    const uint16_t *src_s = p.scales + row * static_cast<size_t>(p.capacity / T) * kHeadDim;
     const int row_tok0 = static_cast<int>(row * p.capacity);
-    const int scan_total = dense ? 0 : nbs;
+    const int scan_total = dense ? 0 : nref + nbs;
     int sc_next = 0;                // scan tiles issued
     int it_next = 0;                // attention stages issued (items + end markers)
     int q_ptr = 0, sub = 0;         // position in the kept-block list
@@ -317,14 +329,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       bool progress = false;
       // scan tiles
       while (sc_next < scan_total) {
+        if (sc_next == 1 && local_in_smem) {  // the attention warps build this tile
+          ++sc_next;
+          continue;
+        }
         const int st = sc_next % NSA;
         const int use = sc_next / NSA;
         if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
+        const int jb = scan_block_index(sc_next, nref, nb, j0);
         uint8_t *dst = scan_ring + st * SG::kStageBytes;
         mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
-        bulk_g2s(dst, src_p + static_cast<size_t>(sc_next) * T * kPackedRowBytes,
-                 T * kPackedRowBytes, &full_a[st]);
-        bulk_g2s(dst + T * kPackedRowBytes, src_s + static_cast<size_t>(sc_next) * kHeadDim,
+        bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * kPackedRowBytes, T * kPackedRowBytes,
+                 &full_a[st]);
+        bulk_g2s(dst + T * kPackedRowBytes, src_s + static_cast<size_t>(jb) * kHeadDim,
                  kScaleRowBytes, &full_a[st]);
         ++sc_next;
         progress = true;
@@ -385,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         __nanosleep(32);
       }
     }
-    drain_ring(full_a, NSA, sc_next);
+    drain_ring(full_a, NSA, sc_next);  // (a skipped entry's phase is completed by its builders)
     drain_ring(full_b, kKvStagesN, it_next);
     return;
   }
@@ -413,18 +430,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     float run0 = -INFINITY, run1 = -INFINITY;  // running max of heads 2*t4, 2*t4 + 1
     int qn = 0;
-    for (int i = 0; i < nbs; ++i) {
-      const int st = i % NSA;
-      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(i / NSA) & 1u, kWaitLimitNs)) {
+    for (int e = 0; e < nref + nbs; ++e) {
+      const int st = e % NSA;
+      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, kWaitLimitNs)) {
         raise_timeout(p, ctrl);
         break;
       }
+      const int jb = scan_block_index(e, nref, nb, j0);
       const uint8_t *tile = scan_ring + st * SG::kStageBytes;
       float s0, s1;
       scan_block<T, G>(tile, reinterpret_cast<const uint16_t *>(tile + T * kPackedRowBytes), qreg,
-                       min(T, len - (j0 + i) * T), lane, s0, s1);
+                       min(T, len - jb * T), lane, s0, s1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_a[st]);
+      if (e < nref) {  // reference blocks: the split's running max starts at their max
+        run0 = fmaxf(run0, s0);
+        run1 = fmaxf(run1, s1);
+        continue;
+      }
+      const int i = e - nref;
       // Top-delta against the running maximum of the split, union over the group
       bool keep = false;
       if (gid == 0) {
@@ -469,6 +493,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       qb[ks][0] = gid < G ? qh[8 * ks + t4] : 0u;
       qb[ks][1] = gid < G ? qh[8 * ks + 4 + t4] : 0u;
     }
+  }
+  if (local_in_smem) {
+    // Quantise the local block from K into scan stage 1 (the producer skips
+    // that entry); scratch in the attention ring, idle until a block is kept,
+    // which cannot happen before this entry has been scanned.
+    const int jl = nb - 1;
+    uint8_t *tile = scan_ring + 1 * SG::kStageBytes;
+    float *red = reinterpret_cast<float *>(kv_ring);
+    quantize_block<T, kAttnThreads>(p.k + (row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T) * kHeadDim,
+                                    min(T, len - jl * T), tile,
+                                    reinterpret_cast<uint16_t *>(tile + T * kPackedRowBytes), red,
+                                    red + (kAttnThreads / 32) * kHeadDim, static_cast<int>(threadIdx.x), 2);
+    fence_proxy_async_smem();  // both regions are later written by async copies
+    named_barrier(2, kAttnThreads);
+    if (threadIdx.x == 0) mbar_arrive(&full_a[1]);
   }
   float m_run[2] = {-INFINITY, -INFINITY};  // heads 2*t4, 2*t4 + 1
   float l_run[2] = {0.0f, 0.0f};
@@ -671,9 +710,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float *ps = row_parts + (s * G + h) * kPartialStride;
       const float ms = __ldcg(ps + 128), ls = __ldcg(ps + 129);
       if (s < chunk) wts[s * G + h] = ms;
-      const float mn = fmaxf(m, ms);  // ms is finite: every split keeps a valid token
-      l = l * exp2f(m - mn) + ls * exp2f(ms - mn);
-      m = mn;
+      const float mn = fmaxf(m, ms);  // -inf only while no split so far kept a token
+      if (mn != -INFINITY) {
+        l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (ms == -INFINITY ? 0.0f : ls * exp2f(ms - mn));
+        m = mn;
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -697,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = threadIdx.x; i < cnt * G; i += kAttnThreads) {
       const int h = i % G, s = s0 + i / G;
       const float ms = s0 == 0 ? wts[i] : __ldcg(row_parts + (s * G + h) * kPartialStride + 128);
-      wts[i] = exp2f(ms - stats[2 * h]) / stats[2 * h + 1];
+      wts[i] = ms == -INFINITY ? 0.0f : exp2f(ms - stats[2 * h]) / stats[2 * h + 1];
     }
     named_barrier(1, kAttnThreads);
 #pragma unroll

@@ -39,6 +39,9 @@ struct DecodeParams {
   int32_t dense;
   // fused decode step: re-quantise each sequence's last key block first
   int32_t requant_last;
+  // reference maximum: 0 = running max inside the split, 1 = pseudo-max from
+  // the sink (first) and local (last) blocks
+  int32_t reference;
   const uint16_t *k;         // bf16 [B][Hkv][cap][D] (read by the re-quantisation)
   uint8_t *packed_out;       // = packed, written for the last block
   uint16_t *scales_out;      // = scales, written for the last block

@@ -33,7 +33,11 @@ EXPORTED = (
     "ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words", "ffd_decode_workspace_bytes",
     "ffd_workspace_init", "ffd_quantize_keys", "ffd_decode", "ffd_check_device_status",
     "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc", "ffd_decode_step",
+    "ffd_decode_ex",
 )
+
+FFD_REFERENCE_RUNNING_MAX = 0
+FFD_REFERENCE_SINK_LOCAL = 1
 
 # Size of the library's built-in scratch array used by ffd_decode_no_alloc.
 FFD_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -43,6 +47,10 @@ class FFDError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class DecodeOptions(ctypes.Structure):
+    _fields_ = [("reference", ctypes.c_int32), ("requant_last", ctypes.c_int32)]
 
 
 class Shape(ctypes.Structure):
@@ -88,6 +96,9 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_quantize_keys.restype = st
             lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode.restype = st
+            lib.ffd_decode_ex.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p,
+                                          ctypes.c_float, p, p, p, sz, p]
+            lib.ffd_decode_ex.restype = st
             lib.ffd_decode_step.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode_step.restype = st
             lib.ffd_decode_no_alloc.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p]
@@ -181,6 +192,18 @@ def decode_step(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float
                                            float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(),
                                            _stream(stream)), "ffd_decode_step")
+
+
+def decode_ex(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out, mask,
+              workspace, reference: int = FFD_REFERENCE_RUNNING_MAX, requant_last: bool = False,
+              stream=None) -> None:
+    """ffd_decode / ffd_decode_step with the reference-maximum mode."""
+    opts = DecodeOptions(int(reference), 1 if requant_last else 0)
+    _check(load_library().ffd_decode_ex(ctypes.byref(shape), ctypes.byref(opts), _ptr(q), _ptr(k),
+                                         _ptr(v), _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
+                                         float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)), "ffd_decode_ex")
 
 
 def decode_no_alloc(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out,

@@ -118,6 +118,11 @@ def test_bad_arguments_rejected_on_host():
                                None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_decode_step(ctypes.byref(s), a, a, a, a, a, a, -1.0, a, a, a, ws,
                                None) == ffd.FFD_ERR_INVALID_ARG
+    for bad in (ffd.DecodeOptions(2, 0), ffd.DecodeOptions(-1, 0), ffd.DecodeOptions(0, 2)):
+        assert lib.ffd_decode_ex(ctypes.byref(s), ctypes.byref(bad), a, a, a, a, a, a, 1.0, a, a,
+                                 a, ws, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_decode_ex(ctypes.byref(s), None, a, a, a, a, a, a, 1.0, a, a, a, ws,
+                             None) == ffd.FFD_ERR_INVALID_ARG
 
 
 def test_product_path_never_touches_the_oracle():

@@ -274,3 +274,89 @@ def test_decode_step_equals_quantize_then_decode(T, delta):
     assert_mask_equal(a.bufs.mask.cpu().numpy().view(np.uint32), want_mask, f"step T{T} {delta}")
     assert_output_close(bf16_to_np_f32(a.bufs.out).astype(np.float64), want_out, f"step T{T} {delta}")
     assert ffd.check_device_status(a.bufs.workspace) == 0
+
+
+# ------------------------------------- pseudo-max reference (sink + local) --
+
+@pytest.mark.parametrize("delta", [0.0, 0.75, 2.0, INF])
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c[0]}")
+def test_decode_pseudo_max_small(case, delta):
+    w, inp = _small(case)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales,
+                                           inp["lengths"], w.block_size, w.split_blocks, delta,
+                                           pseudo_max=True)
+    gc = GpuCase(w, inp)
+    gc.quantize(0)
+    ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
+                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace,
+                  reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+    torch.cuda.synchronize()
+    from gpu_util import bf16_to_np_f32
+    mask = gc.bufs.mask.cpu().numpy().view(np.uint32)
+    assert_mask_equal(mask, want_mask, f"pseudo case {case[0]} delta {delta}")
+    assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out,
+                        f"pseudo case {case[0]} delta {delta}")
+    assert ffd.check_device_status(gc.bufs.workspace) == 0
+
+
+@pytest.mark.parametrize("T,delta", [(64, 0.5), (128, 1.5)])
+def test_decode_step_pseudo_max_equals_quantize_then_decode(T, delta):
+    # several splits per sequence, so CTAs that do not own the last block
+    # build its int4 tile themselves while the owner rewrites it
+    w = fw.random_small_workload(60 + T, 3, 4, 2, 32 * T, T, 3, 2.0, 12 * T, 32 * T, needles=2)
+    inp = fw.make_inputs(w)
+    final = inp["lengths"].copy()
+    a = GpuCase(w, inp, lengths=final - 4)
+    b = GpuCase(w, inp, lengths=final - 4)
+    a.quantize(0)
+    b.quantize(0)
+    for step in range(4):
+        ln = torch.from_numpy(final - 3 + step).cuda()
+        a.lengths.copy_(ln)
+        b.lengths.copy_(ln)
+        ffd.decode_ex(a.shape, a.q, a.k, a.v, a.bufs.k_packed, a.bufs.k_scales, a.lengths, delta,
+                      a.bufs.out, a.bufs.mask, a.bufs.workspace,
+                      reference=ffd.FFD_REFERENCE_SINK_LOCAL, requant_last=True)
+        b.quantize(ffd.FFD_LAST_BLOCK)
+        ffd.decode_ex(b.shape, b.q, b.k, b.v, b.bufs.k_packed, b.bufs.k_scales, b.lengths, delta,
+                      b.bufs.out, b.bufs.mask, b.bufs.workspace,
+                      reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+        torch.cuda.synchronize()
+        assert torch.equal(a.bufs.out.view(torch.int16), b.bufs.out.view(torch.int16))
+        assert torch.equal(a.bufs.mask, b.bufs.mask)
+        assert torch.equal(a.bufs.k_packed, b.bufs.k_packed)
+        assert torch.equal(a.bufs.k_scales.view(torch.int16), b.bufs.k_scales.view(torch.int16))
+    packed, scales = oracle.quantize_keys(inp["k"], final, w.block_size)
+    want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales, final,
+                                           w.block_size, w.split_blocks, delta, pseudo_max=True)
+    from gpu_util import bf16_to_np_f32
+    assert_mask_equal(a.bufs.mask.cpu().numpy().view(np.uint32), want_mask, "pseudo step")
+    assert_output_close(bf16_to_np_f32(a.bufs.out).astype(np.float64), want_out, "pseudo step")
+
+
+@pytest.mark.parametrize("name,delta", [("long128k", 3.0), ("max256k", 1.0), ("ragged", 3.0)])
+def test_full_config_pseudo_max(name, delta):
+    w = fw.WORKLOADS[name]
+    inp = fw.make_inputs(w)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+    _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
+                                 w.split_blocks, delta, pseudo_max=True)
+    want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
+                                w.block_size)
+    gc = GpuCase(w, inp)
+    gc.quantize(0)
+    ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
+                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace,
+                  reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+    torch.cuda.synchronize()
+    from gpu_util import bf16_to_np_f32
+    mask = gc.bufs.mask.cpu().numpy().view(np.uint32)
+    assert_mask_equal(mask, want_mask, f"{name} pseudo")
+    mx, mean = assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out,
+                                   f"{name} pseudo")
+    nblk = w.capacity // w.block_size
+    kept = sum(int(oracle.mask_to_blocks(mask[b, g], nblk).sum())
+               for b in range(w.batch) for g in range(w.num_kv_heads))
+    print(name, "pseudo-max kept", kept, "max-abs", mx, "mean-abs", mean)
