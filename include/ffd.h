@@ -182,6 +182,34 @@ ffd_status ffd_decode_ex(const ffd_shape *shape, const ffd_decode_options *optio
                          void *k_scales, const int32_t *d_lengths, float delta, void *out_bf16,
                          uint32_t *mask, void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* Context (sequence) sharding across GPUs.  Each rank holds a contiguous
+ * shard of every sequence's cache: rank r holds global tokens
+ * [r * cap_local, (r + 1) * cap_local) in a cache of capacity cap_local, with
+ * cap_local a multiple of block_size * split_blocks so that every split lies
+ * in one shard and its Top-delta selection is exactly the unsharded one
+ * (running-max reference only: the pseudo-max needs the sink and local blocks
+ * of other shards).  Steps per decode step:
+ *   1. ffd_decode_partials on every rank with the LOCAL shape and the local
+ *      lengths clip(len - r * cap_local, 0, cap_local): writes the shard's
+ *      split partials and selection bits into its workspace (no merge, no
+ *      output);
+ *   2. all-gather the workspace region named by ffd_partials_region (same
+ *      offset and size on every rank) into num_shards consecutive regions;
+ *   3. ffd_merge_partials with the global lengths: the log-sum-exp merge over
+ *      every split of every shard, writing out [B][Hq][D] and the mask over the
+ *      global capacity num_shards * cap_local ([B][Hkv][ceil(nblk_global/32)]).
+ * Both kernels are the flash-decoding split merge stretched across GPUs; the
+ * exchange moves B * Hkv * nsplit * G * 528 bytes plus the bits per rank. */
+ffd_status ffd_decode_partials(const ffd_shape *local_shape, const ffd_decode_options *options,
+                               const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                               void *k_packed, void *k_scales, const int32_t *d_local_lengths,
+                               float delta, void *workspace, size_t workspace_bytes,
+                               void *cuda_stream);
+ffd_status ffd_partials_region(const ffd_shape *local_shape, size_t *offset, size_t *bytes);
+ffd_status ffd_merge_partials(const ffd_shape *local_shape, int32_t num_shards, const void *gathered,
+                              size_t gathered_bytes, const int32_t *d_global_lengths,
+                              void *out_bf16, uint32_t *mask, void *cuda_stream);
+
 /* ffd_decode without a caller workspace, for callers that cannot allocate
  * device memory: e.g. a plug-in inside an inference engine that is given only
  * its input and output buffers, or a serving loop that must not call

@@ -187,11 +187,17 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
                          const void *v_bf16, const void *k_packed, const void *k_scales,
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
-                         int32_t reference) {
+                         int32_t reference, bool partials_only = false) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL)
     return FFD_ERR_INVALID_ARG;
+  if (partials_only) {
+    // a context shard: splits must not straddle shards, and the pseudo-max
+    // would need the sink and local blocks of other shards
+    if (s->capacity % (s->block_size * s->split_blocks) != 0) return FFD_ERR_INVALID_ARG;
+    if (reference != FFD_REFERENCE_RUNNING_MAX) return FFD_ERR_UNSUPPORTED;
+  }
   if (std::isnan(delta) || delta < 0.0f) return FFD_ERR_INVALID_ARG;
   if (s->batch == 0) return FFD_OK;
   const bool dense = std::isinf(delta);
@@ -200,13 +206,13 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
       workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks);
   if (workspace == nullptr || workspace_bytes < L.total) return FFD_ERR_WORKSPACE;
   if (q_bf16 == nullptr || k_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
-      out_bf16 == nullptr || mask == nullptr)
+      (!partials_only && (out_bf16 == nullptr || mask == nullptr)))
     return FFD_ERR_INVALID_ARG;
   const bool need_packed = requant || !dense;
   if (need_packed && (k_packed == nullptr || k_scales == nullptr)) return FFD_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
       !aligned16(mask) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
-    return FFD_ERR_INVALID_ARG;
+    return FFD_ERR_INVALID_ARG;  // (null out/mask pass: aligned16(nullptr) holds)
   if (need_packed && (!aligned16(k_packed) || !aligned16(k_scales))) return FFD_ERR_INVALID_ARG;
 
   const uint64_t rows = static_cast<uint64_t>(s->batch) * s->num_kv_heads * s->capacity;
@@ -237,6 +243,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
   p.dense = dense ? 1 : 0;
   p.requant_last = requant ? 1 : 0;
   p.reference = reference;
+  p.partials_only = partials_only ? 1 : 0;
   p.k = static_cast<const uint16_t *>(k_bf16);
   p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(k_packed)) : nullptr;
   p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(k_scales)) : nullptr;
@@ -266,6 +273,68 @@ ffd_status ffd_decode_step(const ffd_shape *s, const void *q_bf16, const void *k
                            void *workspace, size_t workspace_bytes, void *cuda_stream) {
   return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, true, FFD_REFERENCE_RUNNING_MAX);
+}
+
+ffd_status ffd_decode_partials(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,
+                               const void *k_bf16, const void *v_bf16, void *k_packed, void *k_scales,
+                               const int32_t *d_local_lengths, float delta, void *workspace,
+                               size_t workspace_bytes, void *cuda_stream) {
+  if (opt == nullptr || (opt->requant_last != 0 && opt->requant_last != 1)) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_local_lengths, delta, nullptr,
+                       nullptr, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
+                       opt->reference, true);
+}
+
+ffd_status ffd_partials_region(const ffd_shape *s, size_t *offset, size_t *bytes) {
+  ffd_status st = check_shape(s);
+  if (st != FFD_OK) return st;
+  if (offset == nullptr || bytes == nullptr) return FFD_ERR_INVALID_ARG;
+  const WorkspaceLayout L = workspace_layout(s->batch, s->num_kv_heads, s->num_q_heads / s->num_kv_heads,
+                                             s->capacity, s->block_size, s->split_blocks);
+  *offset = L.split_bits;
+  *bytes = L.total - L.split_bits;
+  return FFD_OK;
+}
+
+ffd_status ffd_merge_partials(const ffd_shape *s, int32_t num_shards, const void *gathered,
+                              size_t gathered_bytes, const int32_t *d_global_lengths, void *out_bf16,
+                              uint32_t *mask, void *cuda_stream) {
+  ffd_status st = check_shape(s);
+  if (st != FFD_OK) return st;
+  if (num_shards < 1 || s->capacity % (s->block_size * s->split_blocks) != 0) return FFD_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(num_shards) * s->capacity >= (int64_t{1} << 31)) return FFD_ERR_UNSUPPORTED;
+  if (s->batch == 0) return FFD_OK;
+  const int group = s->num_q_heads / s->num_kv_heads;
+  const WorkspaceLayout L =
+      workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks);
+  const size_t region = L.total - L.split_bits;
+  if (gathered == nullptr || d_global_lengths == nullptr || out_bf16 == nullptr || mask == nullptr)
+    return FFD_ERR_INVALID_ARG;
+  if (gathered_bytes < region * num_shards) return FFD_ERR_WORKSPACE;
+  if (!aligned16(gathered) || !aligned16(out_bf16) || !aligned16(mask) ||
+      (reinterpret_cast<uintptr_t>(d_global_lengths) & 3u) != 0)
+    return FFD_ERR_INVALID_ARG;
+  // split weights of every shard live in shared memory (48 KiB without opt-in)
+  if ((16 + static_cast<int64_t>(num_shards) * L.nsplit_max * group) * 4 > 48 * 1024)
+    return FFD_ERR_UNSUPPORTED;
+  MergeParams p{};
+  p.gathered = static_cast<const uint8_t *>(gathered);
+  p.region_bytes = region;
+  p.partials_offset = L.partials - L.split_bits;
+  p.lengths = d_global_lengths;
+  p.out = static_cast<uint16_t *>(out_bf16);
+  p.mask = mask;
+  p.num_kv_heads = s->num_kv_heads;
+  p.capacity = s->capacity;
+  p.split_blocks = s->split_blocks;
+  p.nsplit_max = L.nsplit_max;
+  p.split_words = L.split_words;
+  p.mask_words = static_cast<int32_t>((static_cast<int64_t>(num_shards) * (s->capacity / s->block_size) + 31) / 32);
+  p.num_shards = num_shards;
+  const dim3 grid(static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
+  if (launch_merge(p, s->block_size, group, grid, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+    return FFD_ERR_CUDA;
+  return FFD_OK;
 }
 
 ffd_status ffd_decode_ex(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,

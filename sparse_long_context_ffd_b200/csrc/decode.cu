@@ -257,8 +257,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // Empty or invalid sequence: split 0 writes zero rows and an empty mask.
     if (split == 0) {
       if (bad && threadIdx.x == 0 && g == 0) atomicOr(p.err, kFlagBadLength);
-      for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) out_rows[i] = 0;
-      for (int w = threadIdx.x; w < p.mask_words; w += blockDim.x) p.mask[row * p.mask_words + w] = 0u;
+      if (!p.partials_only) {  // (a context shard leaves the rows to the merge)
+        for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) out_rows[i] = 0;
+        for (int w = threadIdx.x; w < p.mask_words; w += blockDim.x) p.mask[row * p.mask_words + w] = 0u;
+      }
     }
     return;
   }
@@ -681,6 +683,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     p.split_bits[unit * p.split_words + threadIdx.x] = bits;
   }
+  if (p.partials_only) return;  // context shard: the merge runs after the exchange
   __threadfence();
   named_barrier(1, kAttnThreads);
   if (threadIdx.x == 0)

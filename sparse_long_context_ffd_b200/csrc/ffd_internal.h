@@ -45,6 +45,20 @@ struct DecodeParams {
   const uint16_t *k;         // bf16 [B][Hkv][cap][D] (read by the re-quantisation)
   uint8_t *packed_out;       // = packed, written for the last block
   uint16_t *scales_out;      // = scales, written for the last block
+  // context sharding: write the split partials and bits only (no final merge;
+  // out and mask unused)
+  int32_t partials_only;
+};
+
+// Merge of split partials gathered from num_shards context shards.
+struct MergeParams {
+  const uint8_t *gathered;  // num_shards x region_bytes
+  size_t region_bytes;      // one shard's workspace region: split bits, then partials
+  size_t partials_offset;   // offset of the partials inside a region
+  const int32_t *lengths;   // global lengths [B]
+  uint16_t *out;            // bf16 [B][Hq][D]
+  uint32_t *mask;           // [B][Hkv][mask_words] over the global capacity
+  int32_t num_kv_heads, capacity, split_blocks, nsplit_max, split_words, mask_words, num_shards;
 };
 
 struct QuantizeParams {
@@ -66,6 +80,8 @@ WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t gr
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks);
 
+cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 grid,
+                         cudaStream_t stream);
 cudaError_t launch_quantize(const QuantizeParams &p, int block_size, dim3 grid,
                             cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k,

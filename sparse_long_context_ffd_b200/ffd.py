@@ -33,7 +33,7 @@ EXPORTED = (
     "ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words", "ffd_decode_workspace_bytes",
     "ffd_workspace_init", "ffd_quantize_keys", "ffd_decode", "ffd_check_device_status",
     "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc", "ffd_decode_step",
-    "ffd_decode_ex",
+    "ffd_decode_ex", "ffd_decode_partials", "ffd_partials_region", "ffd_merge_partials",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -99,6 +99,13 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_decode_ex.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p,
                                           ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode_ex.restype = st
+            lib.ffd_decode_partials.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p,
+                                                p, ctypes.c_float, p, sz, p]
+            lib.ffd_decode_partials.restype = st
+            lib.ffd_partials_region.argtypes = [sp, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+            lib.ffd_partials_region.restype = st
+            lib.ffd_merge_partials.argtypes = [sp, ctypes.c_int32, p, sz, p, p, p, p]
+            lib.ffd_merge_partials.restype = st
             lib.ffd_decode_step.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode_step.restype = st
             lib.ffd_decode_no_alloc.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p]
@@ -204,6 +211,36 @@ def decode_ex(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, 
                                          float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(),
                                          _stream(stream)), "ffd_decode_ex")
+
+
+def decode_partials(local_shape: Shape, q, k, v, k_packed, k_scales, local_lengths,
+                    delta: float, workspace, requant_last: bool = False, stream=None) -> None:
+    """Context shard: split partials and bits into the workspace, no merge."""
+    opts = DecodeOptions(FFD_REFERENCE_RUNNING_MAX, 1 if requant_last else 0)
+    _check(load_library().ffd_decode_partials(ctypes.byref(local_shape), ctypes.byref(opts),
+                                               _ptr(q), _ptr(k), _ptr(v), _ptr(k_packed),
+                                               _ptr(k_scales), _ptr(local_lengths), float(delta),
+                                               _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(),
+                                               _stream(stream)), "ffd_decode_partials")
+
+
+def partials_region(local_shape: Shape):
+    """(offset, bytes) of the workspace region the shards exchange."""
+    off, nbytes = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(load_library().ffd_partials_region(ctypes.byref(local_shape), ctypes.byref(off),
+                                               ctypes.byref(nbytes)), "ffd_partials_region")
+    return int(off.value), int(nbytes.value)
+
+
+def merge_partials(local_shape: Shape, num_shards: int, gathered, global_lengths, out, mask,
+                   stream=None) -> None:
+    """Merge the gathered shard regions into the output rows and global mask."""
+    _check(load_library().ffd_merge_partials(ctypes.byref(local_shape), int(num_shards),
+                                              _ptr(gathered),
+                                              gathered.numel() * gathered.element_size(),
+                                              _ptr(global_lengths), _ptr(out), _ptr(mask),
+                                              _stream(stream)), "ffd_merge_partials")
 
 
 def decode_no_alloc(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out,

@@ -1,0 +1,48 @@
+"""Context (sequence) sharding of the decode step across GPUs.
+
+Rank r of W holds global tokens [r * cap_local, (r + 1) * cap_local) of every
+sequence; cap_local is a multiple of block_size * split_blocks, so every
+split lies in one shard and its Top-delta selection equals the unsharded one.
+A step is: ffd_decode_partials on the local shard, an all-gather of the
+partials region over NCCL (NVLink / NVSwitch), and ffd_merge_partials.  The
+exchange is B * Hkv * nsplit * G * 528 bytes per rank, so sharding pays only
+when a single GPU's step is long (about 1M tokens and more).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import ffd
+
+
+def local_lengths(global_lengths, rank: int, cap_local: int) -> np.ndarray:
+    """Valid tokens of each sequence in shard `rank`."""
+    g = np.asarray(global_lengths, dtype=np.int64)
+    return np.clip(g - rank * cap_local, 0, cap_local).astype(np.int32)
+
+
+def check_shard_capacity(cap_local: int, block_size: int, split_blocks: int) -> None:
+    if cap_local <= 0 or cap_local % (block_size * split_blocks) != 0:
+        raise ValueError("the shard capacity must be a positive multiple of "
+                         "block_size * split_blocks (shards start at split boundaries)")
+
+
+def global_mask_words(num_shards: int, cap_local: int, block_size: int) -> int:
+    return (num_shards * (cap_local // block_size) + 31) // 32
+
+
+def sharded_decode(local_shape, q, k_local, v_local, packed_local, scales_local,
+                   local_lengths_dev, global_lengths_dev, delta: float, out, mask_global,
+                   workspace, group=None, requant_last: bool = False) -> None:
+    """One decode step over context shards (one rank per GPU, NCCL group)."""
+    import torch
+    import torch.distributed as dist
+    check_shard_capacity(local_shape.capacity, local_shape.block_size, local_shape.split_blocks)
+    world = dist.get_world_size(group)
+    ffd.decode_partials(local_shape, q, k_local, v_local, packed_local, scales_local,
+                        local_lengths_dev, delta, workspace, requant_last=requant_last)
+    off, nbytes = ffd.partials_region(local_shape)
+    region = workspace[off:off + nbytes]
+    gathered = torch.empty(world * nbytes, dtype=torch.uint8, device=workspace.device)
+    dist.all_gather_into_tensor(gathered, region, group=group)
+    ffd.merge_partials(local_shape, world, gathered, global_lengths_dev, out, mask_global)

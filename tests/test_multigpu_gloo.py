@@ -10,6 +10,7 @@ import torch.multiprocessing as mp
 
 import bench
 import ffd_workloads as fw
+import oracle
 
 
 def _free_port():
@@ -71,3 +72,100 @@ def test_algorithmic_bytes_accounting():
     mask[0, 0, 0] = 0b1001  # blocks 0 and 3 (3 holds tokens 192..199)
     kb, vb, kt = bench.kept_tokens_from_mask(w2, np.array([200]), mask)
     assert (kb, vb, kt) == (2, 4, 64 + 8)
+
+
+# ------------------------------------------------ context sharding (host) --
+
+def _partials_numpy(q, k, v, mask_blocks, lengths_local, T, S, G):
+    """Per-split softmax partials (m in base 2, l, acc) of one shard, computed
+    from the selected blocks -- the quantity ffd_decode_partials exchanges."""
+    B, Hq, D = q.shape
+    nsplit = -(-(k.shape[2] // T) // S)
+    m = np.full((B, Hq, nsplit), -np.inf)
+    l = np.zeros((B, Hq, nsplit))
+    acc = np.zeros((B, Hq, nsplit, D))
+    qf = fw.bf16_bits_to_f32(q).astype(np.float64)
+    kf = fw.bf16_bits_to_f32(k).astype(np.float64)
+    vf = fw.bf16_bits_to_f32(v).astype(np.float64)
+    for b in range(B):
+        n = int(lengths_local[b])
+        for h in range(Hq):
+            g = h // G
+            for t in range(n):
+                j = t // T
+                if not mask_blocks[b, g, j]:
+                    continue
+                s = j // S
+                x = qf[b, h] @ kf[b, g, t] / np.sqrt(D) * np.log2(np.e)
+                mn = max(m[b, h, s], x)
+                scale = 0.0 if m[b, h, s] == -np.inf else 2.0 ** (m[b, h, s] - mn)
+                l[b, h, s] = l[b, h, s] * scale + 2.0 ** (x - mn)
+                acc[b, h, s] = acc[b, h, s] * scale + 2.0 ** (x - mn) * vf[b, g, t]
+                m[b, h, s] = mn
+    return m, l, acc
+
+
+def _shard_worker(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    from sparse_long_context_ffd_b200 import sharded
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.dist_init("gloo", world)
+    try:
+        T, S, G, Hkv, B = 64, 2, 2, 1, 2
+        cap_local = T * S * 2
+        cap = world * cap_local
+        w = fw.Workload("shard", B, G * Hkv, Hkv, cap, T, S, 1.0, 5, ragged=(cap_local // 2, cap),
+                        needles=1)
+        inp = fw.make_inputs(w)  # every rank draws the same global inputs
+        lengths = inp["lengths"]
+        packed, scales = oracle.quantize_keys(inp["k"], lengths, T)
+        sc = oracle.block_scores(inp["q"], packed, scales, lengths, T)
+        _, gmask = oracle.select(sc, lengths, Hkv, cap, T, S, 1.0)
+        nblk = cap // T
+        blocks = np.array([[oracle.mask_to_blocks(gmask[b, g], nblk) for g in range(Hkv)]
+                           for b in range(B)])
+        sharded.check_shard_capacity(cap_local, T, S)
+        ll = sharded.local_lengths(lengths, rank, cap_local)
+        sl = slice(rank * cap_local, (rank + 1) * cap_local)
+        m, l, acc = _partials_numpy(inp["q"], inp["k"][:, :, sl], inp["v"][:, :, sl],
+                                    blocks[:, :, rank * (cap_local // T):(rank + 1) * (cap_local // T)],
+                                    ll, T, S, G)
+        mine = torch.from_numpy(np.concatenate([m.ravel(), l.ravel(), acc.ravel()]))
+        gathered = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(gathered, mine)
+        # log-sum-exp merge over every split of every shard
+        parts = []
+        for t in gathered:
+            a = t.numpy()
+            n1 = m.size
+            parts.append((a[:n1].reshape(m.shape), a[n1:2 * n1].reshape(m.shape),
+                          a[2 * n1:].reshape(acc.shape)))
+        M = np.max(np.stack([p[0].max(axis=2) for p in parts]), axis=0)
+        L = sum((p[1] * np.exp2(np.where(np.isinf(p[0]), -np.inf, p[0] - M[..., None]))).sum(axis=2)
+                for p in parts)
+        O = sum((p[2] * np.exp2(np.where(np.isinf(p[0]), -np.inf, p[0] - M[..., None]))[..., None]).sum(axis=2)
+                for p in parts) / L[..., None]
+        want, _ = oracle.attend(inp["q"], inp["k"], inp["v"], lengths, gmask, T)
+        out[rank] = float(np.abs(O - want).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_context_sharding_reproduces_unsharded_attention():
+    world = 2
+    port = _free_port()
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    assert out[0] < 1e-9 and out[1] < 1e-9
+
+
+def test_shard_bookkeeping():
+    from sparse_long_context_ffd_b200 import sharded
+    ll = [sharded.local_lengths([0, 100, 256, 700], r, 256) for r in range(3)]
+    assert [list(x) for x in ll] == [[0, 100, 256, 256], [0, 0, 0, 256], [0, 0, 0, 188]]
+    with pytest.raises(ValueError):
+        sharded.check_shard_capacity(300, 64, 2)
+    assert sharded.global_mask_words(3, 256, 64) == 1
