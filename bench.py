@@ -533,6 +533,70 @@ def run_profile(args):
     return 0
 
 
+def run_shard_measure(args):
+    """One rank's share of a W-way context-sharded decode step, on one GPU:
+    the workload is the local shard (global context = W x its capacity);
+    ffd_decode_partials on it, then ffd_merge_partials over W gathered
+    regions (W copies of the local region: the bytes an all-gather delivers).
+    The all-gather itself needs W GPUs and is not timed; its volume is
+    reported."""
+    import torch
+    from sparse_long_context_ffd_b200 import ffd, sharded
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = fw.WORKLOADS[args.workload]
+    if args.delta is not None:
+        w = fw.scaled_workload(w, delta=args.delta)
+    W = args.shards
+    sharded.check_shard_capacity(w.capacity, w.block_size, w.split_blocks)
+    inp = fw.make_inputs(w)
+    rep = Replica(w, inp, device, 1)
+    L = rep.layers[0]
+    bufs = L["bufs"]
+    off, nbytes = ffd.partials_region(rep.shape)
+    gathered = torch.empty(W * nbytes, dtype=torch.uint8, device=device)
+    glen = torch.from_numpy((inp["lengths"].astype(np.int64) + (W - 1) * w.capacity)
+                            .astype(np.int32)).to(device)  # this shard is full in the global view
+    out = torch.empty((w.batch, w.num_q_heads, 128), dtype=torch.bfloat16, device=device)
+    gmask = torch.empty((w.batch, w.num_kv_heads, sharded.global_mask_words(W, w.capacity,
+                         w.block_size)), dtype=torch.int32, device=device)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        ffd.decode_partials(rep.shape, L["q"], L["k"], L["v"], bufs.k_packed, bufs.k_scales,
+                            rep.lengths, w.delta, bufs.workspace, requant_last=True)
+        if ev:
+            ev[1].record()
+        for r in range(W):  # stand-in for the all-gather (not timed below)
+            gathered[r * nbytes:(r + 1) * nbytes].copy_(bufs.workspace[off:off + nbytes])
+        if ev:
+            ev[2].record()
+        ffd.merge_partials(rep.shape, W, gathered, glen, out, gmask)
+        if ev:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize(device)
+    torch.cuda._sleep(int(1e8))
+    for e in evs:
+        step(e)
+    torch.cuda.synchronize(device)
+    part_us = float(np.mean([e[0].elapsed_time(e[1]) for e in evs])) * 1e3
+    merge_us = float(np.mean([e[2].elapsed_time(e[3]) for e in evs])) * 1e3
+    rep.check_flags()
+    print(json.dumps({
+        "metric": "us per context-sharded decode step, one rank (partials + merge; all-gather not timed)",
+        "value": part_us + merge_us, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": False, "mode": "context-shard",
+        "config": {"workload": w.description + f" as 1 of {W} context shards",
+                   "global_context": W * w.capacity},
+        "partials_us": part_us, "merge_us": merge_us,
+        "exchange_bytes_per_rank": nbytes, "gathered_bytes": W * nbytes}), flush=True)
+    return 0
+
+
 def run_gpu(args):
     import torch
     rank, local_rank, world = dist_env()
@@ -673,6 +737,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--reference-budget", type=float, default=150.0)
+    ap.add_argument("--shards", type=int, default=0,
+                    help="time one rank's share of a context-sharded step over this many shards")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps and exit (for ncu)")
     args = ap.parse_args(argv)
@@ -682,6 +748,8 @@ def main(argv=None):
         return run_reference(args)
     if args.profile_steps:
         return run_profile(args)
+    if args.shards:
+        return run_shard_measure(args)
     return run_gpu(args)
 
 

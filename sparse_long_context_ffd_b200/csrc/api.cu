@@ -314,9 +314,8 @@ ffd_status ffd_merge_partials(const ffd_shape *s, int32_t num_shards, const void
   if (!aligned16(gathered) || !aligned16(out_bf16) || !aligned16(mask) ||
       (reinterpret_cast<uintptr_t>(d_global_lengths) & 3u) != 0)
     return FFD_ERR_INVALID_ARG;
-  // split weights of every shard live in shared memory (48 KiB without opt-in)
-  if ((16 + static_cast<int64_t>(num_shards) * L.nsplit_max * group) * 4 > 48 * 1024)
-    return FFD_ERR_UNSUPPORTED;
+  // every shard's split statistics live in shared memory (48 KiB without opt-in)
+  if (merge_smem_bytes(num_shards, L.nsplit_max) > 48 * 1024) return FFD_ERR_UNSUPPORTED;
   MergeParams p{};
   p.gathered = static_cast<const uint8_t *>(gathered);
   p.region_bytes = region;

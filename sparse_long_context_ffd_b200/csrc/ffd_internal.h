@@ -80,6 +80,7 @@ WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t gr
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks);
 
+size_t merge_smem_bytes(int num_shards, int nsplit_max);
 cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 grid,
                          cudaStream_t stream);
 cudaError_t launch_quantize(const QuantizeParams &p, int block_size, dim3 grid,

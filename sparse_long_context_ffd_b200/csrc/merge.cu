@@ -8,7 +8,9 @@
 // partials of all shards are gathered, this kernel merges them per
 // (sequence, kv-head): M = max m, L = sum l 2^(m - M), o = sum acc 2^(m - M) / L
 // -- the flash-decoding split merge, across GPUs -- and assembles the mask
-// over the global capacity.  One CTA of 128 threads per (kv-head, sequence).
+// over the global capacity.  One CTA of 256 threads per (query head,
+// kv-head, sequence): one round of loads for every split's (m, l), then eight
+// thread groups share the partials' float4 loads.
 #include <cuda_bf16.h>
 
 #include "ffd_internal.h"
@@ -17,7 +19,8 @@
 namespace ffd {
 namespace {
 
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
+constexpr int kGroups = kMergeThreads / 32;  // thread groups, each one float4 per lane of a head
 constexpr uint32_t kFullMask = 0xFFFFFFFFu;
 
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
@@ -25,101 +28,111 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// One CTA per (query head h of the group, kv-head g, sequence b).  Warps are
+// thread groups: group q handles partials f = q, q + kGroups, ...; a lane holds
+// four output channels.
 template <int T, int G>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeParams p) {
   extern __shared__ float smem_f[];
-  float *stats = smem_f;    // [G][2]: M*, L*
-  float *wts = smem_f + 16;  // [num_shards * nsplit_max][G]
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int nflat = p.num_shards * p.nsplit_max;
+  float *ms_s = smem_f;                   // [nflat] split maxima (base 2), -inf if absent
+  float *ls_s = ms_s + nflat;             // [nflat] split sums
+  float *stats = ls_s + nflat;            // [2]: M*, L*
+  // [kGroups][32] float4, 16-byte aligned whatever nflat is
+  float4 *red = reinterpret_cast<float4 *>(smem_f + ((2 * nflat + 4 + 3) & ~3));
+  const int h = blockIdx.x % G, g = blockIdx.x / G, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_q_heads = p.num_kv_heads * G;
   const size_t row = static_cast<size_t>(b) * p.num_kv_heads + g;
-  uint16_t *out_rows = p.out + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim;
+  uint16_t *out_row = p.out + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + h) * kHeadDim;
   const int len = p.lengths[b];
   const int global_cap = p.capacity * p.num_shards;
   const int nblk_local = p.capacity / T;
-  if (len <= 0 || len > global_cap) {  // empty (or invalid) sequence: zero rows, empty mask
-    for (int i = threadIdx.x; i < G * kHeadDim; i += kMergeThreads) out_rows[i] = 0;
-    for (int w = threadIdx.x; w < p.mask_words; w += kMergeThreads) p.mask[row * p.mask_words + w] = 0u;
+  if (len <= 0 || len > global_cap) {  // empty (or invalid) sequence: zero row, empty mask
+    for (int i = threadIdx.x; i < kHeadDim; i += kMergeThreads) out_row[i] = 0;
+    if (h == 0)
+      for (int w = threadIdx.x; w < p.mask_words; w += kMergeThreads) p.mask[row * p.mask_words + w] = 0u;
     return;
   }
-  const int nflat = p.num_shards * p.nsplit_max;
-  auto shard_splits = [&](int r) {
-    const int lr = min(max(len - r * p.capacity, 0), p.capacity);
-    const int nbr = (lr + T - 1) / T;
-    return (nbr + p.split_blocks - 1) / p.split_blocks;
-  };
-  auto partial_ptr = [&](int f, int h) {
+  auto partial_ptr = [&](int f) {
     const int r = f / p.nsplit_max, s = f - r * p.nsplit_max;
     return reinterpret_cast<const float *>(p.gathered + r * p.region_bytes + p.partials_offset) +
            ((row * p.nsplit_max + s) * G + h) * kPartialStride;
   };
-  // 1. per head: pairwise (max, sum) combination over every valid split of every shard
-  for (int h = warp; h < G; h += kMergeThreads / 32) {
+  // 1. every split's (m, l) in one round of independent loads; absent or
+  //    empty splits get m = -inf
+  for (int f = threadIdx.x; f < nflat; f += kMergeThreads) {
+    const int r = f / p.nsplit_max, s = f - r * p.nsplit_max;
+    const int lr = min(max(len - r * p.capacity, 0), p.capacity);
+    const int nsr = ((lr + T - 1) / T + p.split_blocks - 1) / p.split_blocks;
     float m = -INFINITY, l = 0.0f;
-    for (int f = lane; f < nflat; f += 32) {
-      const int r = f / p.nsplit_max, s = f - r * p.nsplit_max;
-      float ms = -INFINITY;
-      if (s < shard_splits(r)) {
-        const float *ps = partial_ptr(f, h);
-        ms = __ldcg(ps + 128);
-        const float ls = __ldcg(ps + 129);
-        const float mn = fmaxf(m, ms);
-        if (mn != -INFINITY) {
-          l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (ms == -INFINITY ? 0.0f : ls * exp2f(ms - mn));
-          m = mn;
-        }
-      }
-      wts[f * G + h] = ms;
+    if (s < nsr) {
+      const float *ps = partial_ptr(f);
+      m = __ldcg(ps + 128);
+      l = __ldcg(ps + 129);
     }
+    ms_s[f] = m;
+    ls_s[f] = l;
+  }
+  __syncthreads();
+  // 2. M* = max m, L* = sum l 2^(m - M*) (warp 0, from shared memory)
+  if (warp == 0) {
+    float m = -INFINITY;
+    for (int f = lane; f < nflat; f += 32) m = fmaxf(m, ms_s[f]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float mo = __shfl_xor_sync(kFullMask, m, off), lo = __shfl_xor_sync(kFullMask, l, off);
-      const float mn = fmaxf(m, mo);
-      if (mn != -INFINITY) {
-        l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mn));
-        m = mn;
-      }
-    }
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
+    float l = 0.0f;
+    for (int f = lane; f < nflat; f += 32)
+      if (ms_s[f] != -INFINITY) l += ls_s[f] * exp2f(ms_s[f] - m);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(kFullMask, l, off);
     if (lane == 0) {
-      stats[2 * h] = m;
-      stats[2 * h + 1] = l;
+      stats[0] = m;
+      stats[1] = l;
     }
   }
   __syncthreads();
-  // 2. weights 2^(m - M*) / L*; splits that do not exist or kept nothing get 0
-  for (int i = threadIdx.x; i < nflat * G; i += kMergeThreads) {
-    const int h = i % G;
-    const float ms = wts[i];
-    wts[i] = ms == -INFINITY ? 0.0f : exp2f(ms - stats[2 * h]) / stats[2 * h + 1];
-  }
+  // 3. weights 2^(m - M*) / L* in place of the maxima
+  for (int f = threadIdx.x; f < nflat; f += kMergeThreads)
+    ms_s[f] = ms_s[f] == -INFINITY ? 0.0f : exp2f(ms_s[f] - stats[0]) / stats[1];
   __syncthreads();
-  // 3. each thread accumulates four output channels (float4) of one head
-  for (int fi = threadIdx.x; fi < G * 32; fi += kMergeThreads) {
-    const int h = fi >> 5, c4 = fi & 31;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int f0 = 0; f0 < nflat; f0 += 8) {
-      float4 v[8];
-      float wv[8];
+  // 4. group `warp` accumulates partials f = warp, warp + kGroups, ... ; lane
+  //    holds channels 4*lane .. 4*lane+3
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int f0 = warp; f0 < nflat; f0 += 8 * kGroups) {
+    float4 v[8];
+    float wv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int f = f0 + u;
-        wv[u] = f < nflat ? wts[f * G + h] : 0.0f;
-        v[u] = wv[u] != 0.0f ? __ldcg(reinterpret_cast<const float4 *>(partial_ptr(f, h)) + c4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc.x += wv[u] * v[u].x;
-        acc.y += wv[u] * v[u].y;
-        acc.z += wv[u] * v[u].z;
-        acc.w += wv[u] * v[u].w;
-      }
+    for (int u = 0; u < 8; ++u) {
+      const int f = f0 + u * kGroups;
+      wv[u] = f < nflat ? ms_s[f] : 0.0f;
+      v[u] = wv[u] != 0.0f ? __ldcg(reinterpret_cast<const float4 *>(partial_ptr(f)) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    *reinterpret_cast<uint2 *>(out_rows + h * kHeadDim + 4 * c4) =
-        make_uint2(pack2_bf16(acc.x, acc.y), pack2_bf16(acc.z, acc.w));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc.x += wv[u] * v[u].x;
+      acc.y += wv[u] * v[u].y;
+      acc.z += wv[u] * v[u].z;
+      acc.w += wv[u] * v[u].w;
+    }
   }
-  // 4. mask over the global capacity: global block j lives in shard j / nblk_local
+  red[warp * 32 + lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 o = red[lane];
+#pragma unroll
+    for (int q = 1; q < kGroups; ++q) {
+      const float4 x = red[q * 32 + lane];
+      o.x += x.x;
+      o.y += x.y;
+      o.z += x.z;
+      o.w += x.w;
+    }
+    *reinterpret_cast<uint2 *>(out_row + 4 * lane) = make_uint2(pack2_bf16(o.x, o.y), pack2_bf16(o.z, o.w));
+  }
+  // 5. the mask row (head 0's CTA): global block j lives in shard j / nblk_local
+  if (h != 0) return;
   const int nb = (len + T - 1) / T;
   for (int w = threadIdx.x; w < p.mask_words; w += kMergeThreads) {
     uint32_t bits = 0, cached = 0;
@@ -155,11 +168,17 @@ cudaError_t launch_t(const MergeParams &p, int group, dim3 grid, size_t smem, cu
 
 }  // namespace
 
+size_t merge_smem_bytes(int num_shards, int nsplit_max) {
+  const size_t floats = (2 * static_cast<size_t>(num_shards) * nsplit_max + 4 + 3) & ~static_cast<size_t>(3);
+  return 4 * floats + 16 * kGroups * 32;
+}
+
 cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 grid,
                          cudaStream_t stream) {
-  const size_t smem = 4 * (16 + static_cast<size_t>(p.num_shards) * p.nsplit_max * group);
-  if (block_size == 64) return launch_t<64>(p, group, grid, smem, stream);
-  if (block_size == 128) return launch_t<128>(p, group, grid, smem, stream);
+  const dim3 g(grid.x * group, grid.y);  // one CTA per query head
+  const size_t smem = merge_smem_bytes(p.num_shards, p.nsplit_max);
+  if (block_size == 64) return launch_t<64>(p, group, g, smem, stream);
+  if (block_size == 128) return launch_t<128>(p, group, g, smem, stream);
   return cudaErrorInvalidValue;
 }
 

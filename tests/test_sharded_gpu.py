@@ -15,10 +15,10 @@ from sparse_long_context_ffd_b200 import ffd, sharded
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("W,T,S,G", [(2, 64, 4, 4), (4, 64, 3, 8), (3, 128, 2, 2)])
+@pytest.mark.parametrize("W,T,S,G", [(2, 64, 4, 4), (4, 64, 3, 8), (3, 128, 2, 2), (3, 64, 1, 4)])
 @pytest.mark.parametrize("delta", [0.5, 2.0, float("inf")])
 def test_sharded_decode_matches_unsharded(W, T, S, G, delta):
-    cap_local = T * S * 4
+    cap_local = T * S * (3 if S == 1 else 4)  # S = 1: 3 splits per shard, 9 in all (odd)
     cap = W * cap_local
     B, Hkv = 3, 2
     w = fw.random_small_workload(90 + W, B, G, Hkv, cap, T, S, delta, 1, cap, needles=2)
