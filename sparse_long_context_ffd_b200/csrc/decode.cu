@@ -788,24 +788,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   // mask row: each word gathers 32 consecutive blocks' bits from the split
-  // bit rows, loading each split word once
+  // bit rows
   const uint32_t *row_bits = p.split_bits + row * p.nsplit_max * p.split_words;
-  for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads) {
-    uint32_t bits = 0, cached = 0;
-    int key = -1;
-    for (int k = 0; k < 32; ++k) {
-      const int j = 32 * w + k;
-      if (j >= nb) break;
-      const int s = j / p.split_blocks, i = j - s * p.split_blocks;
-      const int kk = s * p.split_words + (i >> 5);
-      if (kk != key) {
-        cached = __ldcg(row_bits + kk);
-        key = kk;
-      }
-      bits |= ((cached >> (i & 31)) & 1u) << k;
-    }
-    p.mask[row * p.mask_words + w] = bits;
-  }
+  const int split_words = p.split_words;
+  for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads)
+    p.mask[row * p.mask_words + w] = gather_mask_word(
+        w, nb, p.split_blocks, [&](int s, int wd) { return __ldcg(row_bits + s * split_words + wd); });
   if (threadIdx.x == 0) p.counters[row] = 0u;
 }
 

@@ -165,6 +165,35 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// Keep bits of the 32 blocks 32w .. 32w+31 of a row with nb valid blocks,
+// gathered from per-split bit rows: block j is bit (j % S) % 32 of word
+// (j % S) / 32 of split j / S, and load_word(split, word) fetches one word.
+// Walks the blocks incrementally: one division per word, one load per
+// distinct split word (1 per mask word when S is a multiple of 32).
+template <class LoadWord>
+__device__ __forceinline__ uint32_t gather_mask_word(int w, int nb, int S, LoadWord load_word) {
+  int j = 32 * w;
+  if (j >= nb) return 0u;
+  int s = j / S, i = j - s * S;
+  int cw = i >> 5;
+  uint32_t cached = load_word(s, cw);
+  uint32_t bits = 0u;
+  for (int k = 0; k < 32 && j < nb; ++k, ++j) {
+    if ((i >> 5) != cw) {
+      cw = i >> 5;
+      cached = load_word(s, cw);
+    }
+    bits |= ((cached >> (i & 31)) & 1u) << k;
+    if (++i == S) {  // next split
+      ++s;
+      i = 0;
+      cw = 0;
+      if (j + 1 < nb) cached = load_word(s, 0);
+    }
+  }
+  return bits;
+}
+
 // Named barrier over `count` threads (multiple of 32).
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

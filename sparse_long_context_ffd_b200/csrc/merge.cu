@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeParams 
   float *stats = ls_s + nflat;            // [2]: M*, L*
   // [kGroups][32] float4, 16-byte aligned whatever nflat is
   float4 *red = reinterpret_cast<float4 *>(smem_f + ((2 * nflat + 4 + 3) & ~3));
+  const float **part_s = reinterpret_cast<const float **>(red + kGroups * 32);  // [nflat]
   const int h = blockIdx.x % G, g = blockIdx.x / G, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_q_heads = p.num_kv_heads * G;
@@ -66,13 +67,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeParams 
     const int lr = min(max(len - r * p.capacity, 0), p.capacity);
     const int nsr = ((lr + T - 1) / T + p.split_blocks - 1) / p.split_blocks;
     float m = -INFINITY, l = 0.0f;
+    const float *ps = partial_ptr(f);
     if (s < nsr) {
-      const float *ps = partial_ptr(f);
       m = __ldcg(ps + 128);
       l = __ldcg(ps + 129);
     }
     ms_s[f] = m;
     ls_s[f] = l;
+    part_s[f] = ps;
   }
   __syncthreads();
   // 2. M* = max m, L* = sum l 2^(m - M*) (warp 0, from shared memory)
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeParams 
     for (int u = 0; u < 8; ++u) {
       const int f = f0 + u * kGroups;
       wv[u] = f < nflat ? ms_s[f] : 0.0f;
-      v[u] = wv[u] != 0.0f ? __ldcg(reinterpret_cast<const float4 *>(partial_ptr(f)) + lane)
+      v[u] = wv[u] != 0.0f ? __ldcg(reinterpret_cast<const float4 *>(part_s[f]) + lane)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
@@ -134,24 +136,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeParams 
   // 5. the mask row (head 0's CTA): global block j lives in shard j / nblk_local
   if (h != 0) return;
   const int nb = (len + T - 1) / T;
-  for (int w = threadIdx.x; w < p.mask_words; w += kMergeThreads) {
-    uint32_t bits = 0, cached = 0;
-    int key = -1;
-    for (int k = 0; k < 32; ++k) {
-      const int j = 32 * w + k;
-      if (j >= nb) break;
-      const int r = j / nblk_local, jl = j - r * nblk_local;
-      const int s = jl / p.split_blocks, i = jl - s * p.split_blocks;
-      const int kk = r * 65536 + s * p.split_words + (i >> 5);  // cache key
-      if (kk != key) {
-        const uint32_t *bits_r = reinterpret_cast<const uint32_t *>(p.gathered + r * p.region_bytes);
-        cached = __ldcg(bits_r + (row * p.nsplit_max + s) * p.split_words + (i >> 5));
-        key = kk;
-      }
-      bits |= ((cached >> (i & 31)) & 1u) << k;
-    }
-    p.mask[row * p.mask_words + w] = bits;
-  }
+  // shards start at split boundaries, so the global split index j / S is
+  // shard * nsplit_max + the shard's split index
+  (void)nblk_local;
+  auto load_word = [&](int gs, int wd) {
+    const int r = gs / p.nsplit_max, s = gs - r * p.nsplit_max;
+    const uint32_t *bits_r = reinterpret_cast<const uint32_t *>(p.gathered + r * p.region_bytes);
+    return __ldcg(bits_r + (row * p.nsplit_max + s) * p.split_words + wd);
+  };
+  for (int w = threadIdx.x; w < p.mask_words; w += kMergeThreads)
+    p.mask[row * p.mask_words + w] = gather_mask_word(w, nb, p.split_blocks, load_word);
 }
 
 template <int T>
@@ -169,8 +163,9 @@ cudaError_t launch_t(const MergeParams &p, int group, dim3 grid, size_t smem, cu
 }  // namespace
 
 size_t merge_smem_bytes(int num_shards, int nsplit_max) {
-  const size_t floats = (2 * static_cast<size_t>(num_shards) * nsplit_max + 4 + 3) & ~static_cast<size_t>(3);
-  return 4 * floats + 16 * kGroups * 32;
+  const size_t nflat = static_cast<size_t>(num_shards) * nsplit_max;
+  const size_t floats = (2 * nflat + 4 + 3) & ~static_cast<size_t>(3);
+  return 4 * floats + 16 * kGroups * 32 + 8 * nflat;
 }
 
 cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 grid,
