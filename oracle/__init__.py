@@ -57,6 +57,14 @@ def _load():
                                         ctypes.c_float, p, p, p]
             lib.ffdo_decode_pseudo_max.argtypes = lib.ffdo_decode.argtypes
             lib.ffdo_select_pseudo_max.argtypes = lib.ffdo_select.argtypes
+            lib.ffdo_quantize_keys_tr.argtypes = [i, i, i, i, i, p, p, i, p, p, p]
+            lib.ffdo_fold_query_tr.argtypes = [i, p, p, p, p]
+            lib.ffdo_fold_query_tr.restype = None
+            lib.ffdo_block_scores_tr.argtypes = [i, i, i, i, i, i, p, p, p, p, p]
+            lib.ffdo_reconstruct_keys_tr.argtypes = [i, i, i, i, i, p, p, p, p, p]
+            lib.ffdo_attend_tr.argtypes = [i, i, i, i, i, i, p, p, p, p, p, p, p, p, p]
+            lib.ffdo_decode_tr.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p,
+                                           ctypes.c_float, i, p, p, p]
             _lib = lib
     return _lib
 
@@ -171,3 +179,101 @@ def mask_to_blocks(mask_row, nblk):
     """Expand one [words] uint32 mask row into a bool array of nblk blocks."""
     bits = np.unpackbits(np.asarray(mask_row, dtype="<u4").view(np.uint8), bitorder="little")
     return bits[:nblk].astype(bool)
+
+
+# ---- thumbnail + residual key format (2-bit thumbnails, 8-bit residuals) ----
+
+def quantize_keys_tr(k, lengths, block_size, block_begin=0, thumb=None, resid=None, scales=None):
+    """Thumbnail + residual copy of bf16 keys ``k`` [B,Hkv,cap,D]: returns
+    (thumb [B,Hkv,cap,D/4] u8, resid [B,Hkv,cap,D] u8, scales [B,Hkv,nblk,D]
+    bf16 bits), updated in place when given."""
+    k = _c(k, np.uint16)
+    lengths = _c(lengths, np.int32)
+    B, Hkv, cap, D = k.shape
+    if thumb is None:
+        thumb = np.zeros((B, Hkv, cap, D // 4), dtype=np.uint8)
+    if resid is None:
+        resid = np.zeros((B, Hkv, cap, D), dtype=np.uint8)
+    if scales is None:
+        scales = np.zeros((B, Hkv, cap // block_size, D), dtype=np.uint16)
+    assert thumb.flags.c_contiguous and resid.flags.c_contiguous and scales.flags.c_contiguous
+    _check(_load().ffdo_quantize_keys_tr(B, Hkv, cap, D, block_size, _ptr(k), _ptr(lengths),
+                                         int(block_begin), _ptr(thumb), _ptr(resid),
+                                         _ptr(scales)))
+    return thumb, resid, scales
+
+
+def fold_query_tr(q_head, scale_block):
+    q_head = _c(q_head, np.uint16)
+    scale_block = _c(scale_block, np.uint16)
+    qi = np.zeros(q_head.shape[0], dtype=np.int8)
+    c = np.zeros(1, dtype=np.float32)
+    _load().ffdo_fold_query_tr(q_head.shape[0], _ptr(q_head), _ptr(scale_block), _ptr(qi), _ptr(c))
+    return qi, float(c[0])
+
+
+def block_scores_tr(q, thumb, scales, lengths, block_size):
+    q = _c(q, np.uint16)
+    thumb = _c(thumb, np.uint8)
+    scales = _c(scales, np.uint16)
+    lengths = _c(lengths, np.int32)
+    B, Hq, D = q.shape
+    _, Hkv, cap, _ = thumb.shape
+    out = np.empty((B, Hq, cap // block_size), dtype=np.float32)
+    _check(_load().ffdo_block_scores_tr(B, Hq, Hkv, cap, D, block_size, _ptr(q), _ptr(thumb),
+                                        _ptr(scales), _ptr(lengths), _ptr(out)))
+    return out
+
+
+def reconstruct_keys_tr(thumb, resid, scales, lengths, block_size):
+    """The computer's keys k_hat [B,Hkv,cap,D] (float64; zero past the length)."""
+    thumb = _c(thumb, np.uint8)
+    resid = _c(resid, np.uint8)
+    scales = _c(scales, np.uint16)
+    lengths = _c(lengths, np.int32)
+    B, Hkv, cap, D = resid.shape
+    out = np.zeros((B, Hkv, cap, D), dtype=np.float64)
+    _check(_load().ffdo_reconstruct_keys_tr(B, Hkv, cap, D, block_size, _ptr(thumb), _ptr(resid),
+                                            _ptr(scales), _ptr(lengths), _ptr(out)))
+    return out
+
+
+def attend_tr(q, thumb, resid, scales, v, lengths, mask, block_size):
+    """fp64 attention over the selected blocks with reconstructed keys."""
+    q = _c(q, np.uint16)
+    thumb = _c(thumb, np.uint8)
+    resid = _c(resid, np.uint8)
+    scales = _c(scales, np.uint16)
+    v = _c(v, np.uint16)
+    lengths = _c(lengths, np.int32)
+    mask = _c(mask, np.uint32)
+    B, Hq, D = q.shape
+    _, Hkv, cap, _ = v.shape
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    _check(_load().ffdo_attend_tr(B, Hq, Hkv, cap, D, block_size, _ptr(q), _ptr(thumb),
+                                  _ptr(resid), _ptr(scales), _ptr(v), _ptr(lengths), _ptr(mask),
+                                  _ptr(out), _ptr(lse)))
+    return out, lse
+
+
+def decode_tr(q, v, thumb, resid, scales, lengths, block_size, split_blocks, delta,
+              pseudo_max=False):
+    """The whole step on the thumbnail + residual format.  Returns
+    (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores)."""
+    q = _c(q, np.uint16)
+    v = _c(v, np.uint16)
+    thumb = _c(thumb, np.uint8)
+    resid = _c(resid, np.uint8)
+    scales = _c(scales, np.uint16)
+    lengths = _c(lengths, np.int32)
+    B, Hq, D = q.shape
+    _, Hkv, cap, _ = v.shape
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    mask = np.zeros((B, Hkv, mask_words(cap, block_size)), dtype=np.uint32)
+    scores = np.zeros((B, Hq, cap // block_size), dtype=np.float32)
+    _check(_load().ffdo_decode_tr(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(v),
+                                  _ptr(thumb), _ptr(resid), _ptr(scales), _ptr(lengths),
+                                  float(delta), 1 if pseudo_max else 0, _ptr(out), _ptr(mask),
+                                  _ptr(scores)))
+    return out, mask, scores

@@ -32,16 +32,29 @@
  *   R15 pseudo-max reference (optional mode): the sink tokens are block 0,
  *       the local tokens the last block; the split's running maximum starts
  *       at the larger of their two block scores.
+ *   R16 thumbnail + residual key format (optional, the pages' own split of
+ *       the K cache): per block and channel s = bf16(amax / 1.5); 2-bit code
+ *       u = clamp(floor(k / s) + 2, 0, 3) naming the level (u - 1.5) s;
+ *       8-bit residual e = clamp(rint((k / s - (u - 1.5)) * 254), -127, 127);
+ *       the computer's key is k_hat = s (254 u - 381 + e) / 254.
+ *   R17 thumbnail packing: channel 16w + i of a token row sits in 32-bit
+ *       little-endian word w at bit 2 (i / 2) + 16 (i % 2) (even channels of
+ *       the group in the low half, odd ones in the high half); residual byte
+ *       c holds e_c + 128.  Tokens at or past the length are zero bytes.
+ *   R18 thumbnail block score: the query fold of R4, then
+ *       I_t = sum_c qi_c (2 u_c - 3) and score = float(max_t I_t) * (a / 254)
+ *       / sqrt(D), the thumbnail level being (2u - 3) s / 2.
  *
  * Floating point: the selection steps use fp32 with one IEEE operation per
  * step (this file must be built with -ffp-contract=off and without fast-math);
  * the attention over the selected tokens is computed in fp64.
  *
  * Parity status: attention (closed form / library special cases) and selection
- * (brute-force enumeration) are pinned by the tests; the quantiser and the query
- * fold are pinned by closed-form cases and error bounds only, because the pages
- * specify neither (their keys are 2-bit thumbnails) -- "parity unpinned" against
- * the pages for those two formats.
+ * (brute-force enumeration) are pinned by the tests; the quantisers and the
+ * query fold are pinned by hand-worked examples, closed-form cases and error
+ * bounds only, because the pages fix neither the int4 copy (not theirs) nor
+ * the details of their 2-bit + 8-bit split (R16-R18) -- "parity unpinned"
+ * against the pages for both key formats.
  */
 #include <math.h>
 #include <stdint.h>
@@ -300,11 +313,28 @@ int ffdo_select_pseudo_max(int B, int Hq, int Hkv, int cap, int T, int S, const 
 /* ---- step 5: exact attention over the selected blocks (gist.science,
  *      Methodology 3, stage "Fine-Grained Refinement"; R6, R7), fp64 -------- */
 
-/* out[b][h][c] (double).  Optionally lse[b][h] = log sum exp of the selected
- * logits (natural log, logits already divided by sqrt(D)). */
-int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
-                const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                const int32_t *lengths, const uint32_t *mask, double *out, double *lse) {
+/* Where the computer's keys come from: the bf16 cache (the int4 path reads
+ * full-precision K for kept blocks) or the thumbnail + residual pair of R16,
+ * reconstructed per element. */
+typedef struct {
+  const uint16_t *k;      /* bf16 [B][Hkv][cap][D], or NULL */
+  const uint8_t *thumb;   /* R17 [B][Hkv][cap][D/4] */
+  const uint8_t *resid;   /* [B][Hkv][cap][D] */
+  const uint16_t *scales; /* bf16 [B][Hkv][nblk][D] */
+} key_source;
+
+static double thumb_resid_key(const uint8_t *thumb_row, const uint8_t *resid_row, float sf, int c);
+
+static double key_value(const key_source *ks, size_t row, int cap, int D, int T, int t, int c) {
+  if (ks->k) return (double)bf16_to_float(ks->k[(row * (size_t)cap + (size_t)t) * D + c]);
+  size_t tok = row * (size_t)cap + (size_t)t;
+  float sf = bf16_to_float(ks->scales[(row * (size_t)(cap / T) + (size_t)(t / T)) * D + c]);
+  return thumb_resid_key(ks->thumb + tok * (size_t)(D / 4), ks->resid + tok * (size_t)D, sf, c);
+}
+
+static int attend_impl(int B, int Hq, int Hkv, int cap, int D, int T, const uint16_t *q,
+                       const key_source *ks, const uint16_t *v, const int32_t *lengths,
+                       const uint32_t *mask, double *out, double *lse) {
   if (check_shape(B, Hq, Hkv, cap, D, T) != FFDO_OK) return FFDO_BAD_ARG;
   int G = Hq / Hkv, nblk = cap / T, words = (nblk + 31) / 32;
   for (int b = 0; b < B; ++b)
@@ -316,10 +346,10 @@ int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
     int len = lengths[b];
     for (int h = 0; h < Hq; ++h) {
       int g = h / G;
+      size_t row = (size_t)b * Hkv + g;
       const uint16_t *qh = q + ((size_t)b * Hq + h) * D;
-      const uint16_t *kr = k + ((size_t)b * Hkv + g) * (size_t)cap * D;
-      const uint16_t *vr = v + ((size_t)b * Hkv + g) * (size_t)cap * D;
-      const uint32_t *m = mask + ((size_t)b * Hkv + g) * words;
+      const uint16_t *vr = v + row * (size_t)cap * D;
+      const uint32_t *m = mask + row * words;
       double *o = out + ((size_t)b * Hq + h) * D;
       for (int c = 0; c < D; ++c) o[c] = 0.0;
       double mx = -INFINITY;
@@ -329,7 +359,7 @@ int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
         if (!((m[j / 32] >> (j % 32)) & 1u)) continue;
         double dot = 0.0;
         for (int c = 0; c < D; ++c)
-          dot += (double)bf16_to_float(qh[c]) * (double)bf16_to_float(kr[(size_t)t * D + c]);
+          dot += (double)bf16_to_float(qh[c]) * key_value(ks, row, cap, D, T, t, c);
         logit[t] = dot * scale;
         if (logit[t] > mx) mx = logit[t];
         any = 1;
@@ -351,8 +381,16 @@ int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
     }
   }
   free(logit);
-  (void)nblk;
   return FFDO_OK;
+}
+
+/* out[b][h][c] (double).  Optionally lse[b][h] = log sum exp of the selected
+ * logits (natural log, logits already divided by sqrt(D)). */
+int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
+                const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                const int32_t *lengths, const uint32_t *mask, double *out, double *lse) {
+  key_source ks = {k, NULL, NULL, NULL};
+  return attend_impl(B, Hq, Hkv, cap, D, T, q, &ks, v, lengths, mask, out, lse);
 }
 
 /* ---- the whole decode step: scores -> selection -> attention ------------ */
@@ -407,6 +445,213 @@ static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
            ? ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask)
            : ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
   if (rc == FFDO_OK) rc = ffdo_attend(B, Hq, Hkv, cap, D, T, q, k, v, lengths, mask, out, NULL);
+  free(own);
+  return rc;
+}
+
+/* ==== the pages' key format: 2-bit thumbnails + 8-bit residuals ===========
+ * gist.science explainer, Methodology 1: the K cache is split into 2-bit
+ * quantised thumbnails, which the selector scans to estimate scores, and
+ * 8-bit residuals, which together with the thumbnails reconstruct the keys
+ * for the exact computation (Methodology 3, stage "Fine-Grained Refinement":
+ * kept blocks load residuals and values).  Readings R16-R18. */
+
+/* 2-bit code of channel c of a thumbnail token row (R17). */
+static int thumb_code(const uint8_t *row, int c) {
+  const uint8_t *w = row + 4 * (c / 16);
+  uint32_t word = (uint32_t)w[0] | ((uint32_t)w[1] << 8) | ((uint32_t)w[2] << 16) |
+                  ((uint32_t)w[3] << 24);
+  int i = c % 16;
+  return (int)((word >> (2 * (i / 2) + 16 * (i % 2))) & 3u);
+}
+
+static void put_thumb_code(uint8_t *row, int c, int u) {
+  int i = c % 16, bit = 2 * (i / 2) + 16 * (i % 2);
+  row[4 * (c / 16) + bit / 8] |= (uint8_t)(u << (bit % 8));
+}
+
+/* k_hat = s * (254 u - 381 + e) / 254 with e = residual byte - 128 (R16). */
+static double thumb_resid_key(const uint8_t *thumb_row, const uint8_t *resid_row, float sf, int c) {
+  int u = thumb_code(thumb_row, c);
+  int e = (int)resid_row[c] - 128;
+  return (double)sf * (double)(254 * u - 381 + e) / 254.0;
+}
+
+/* Quantise blocks [block_begin, nb_b) (block_begin < 0: the last block only)
+ * of every (b, g) row into thumb [B][Hkv][cap][D/4], resid [B][Hkv][cap][D]
+ * and scales [B][Hkv][nblk][D] (R16, R17). */
+int ffdo_quantize_keys_tr(int B, int Hkv, int cap, int D, int T,
+                          const uint16_t *k, const int32_t *lengths, int block_begin,
+                          uint8_t *thumb, uint8_t *resid, uint16_t *scales) {
+  if (check_shape(B, Hkv, Hkv, cap, D, T) != FFDO_OK) return FFDO_BAD_ARG;
+  int nblk = cap / T;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 0 || lengths[b] > cap) return FFDO_BAD_LENGTH;
+  for (int b = 0; b < B; ++b) {
+    int len = lengths[b];
+    int nb = (len + T - 1) / T;
+    int j0 = block_begin < 0 ? nb - 1 : block_begin;
+    if (j0 < 0) j0 = 0;
+    for (int g = 0; g < Hkv; ++g) {
+      size_t row = (size_t)b * Hkv + g;
+      const uint16_t *krow = k + row * (size_t)cap * D;
+      uint8_t *trow = thumb + row * (size_t)cap * (D / 4);
+      uint8_t *rrow = resid + row * (size_t)cap * D;
+      uint16_t *srow = scales + row * (size_t)nblk * D;
+      for (int j = j0; j < nb; ++j) {
+        int t_end = (j + 1) * T < len ? (j + 1) * T : len;
+        float sf[128];
+        for (int c = 0; c < D; ++c) {
+          float amax = 0.0f;
+          for (int t = j * T; t < t_end; ++t) {
+            float x = fabsf(bf16_to_float(krow[(size_t)t * D + c]));
+            if (x > amax) amax = x;
+          }
+          uint16_t sc = float_to_bf16(amax / 1.5f);
+          srow[(size_t)j * D + c] = sc;
+          sf[c] = bf16_to_float(sc);
+        }
+        for (int t = j * T; t < (j + 1) * T; ++t) {
+          uint8_t *tr = trow + (size_t)t * (D / 4);
+          uint8_t *rr = rrow + (size_t)t * D;
+          memset(tr, 0, (size_t)(D / 4));
+          memset(rr, 0, (size_t)D);
+          if (t >= t_end) continue; /* past the length: zero bytes */
+          for (int c = 0; c < D; ++c) {
+            int u = 2, e = 0;
+            if (sf[c] != 0.0f) {
+              float y = bf16_to_float(krow[(size_t)t * D + c]) / sf[c];
+              float uf = floorf(y) + 2.0f;
+              if (uf < 0.0f) uf = 0.0f;
+              if (uf > 3.0f) uf = 3.0f;
+              u = (int)uf;
+              float d = y - ((float)u - 1.5f);
+              float r = nearbyintf(d * 254.0f);
+              if (r > 127.0f) r = 127.0f;
+              if (r < -127.0f) r = -127.0f;
+              e = (int)r;
+            }
+            put_thumb_code(tr, c, u);
+            rr[c] = (uint8_t)(e + 128);
+          }
+        }
+      }
+    }
+  }
+  return FFDO_OK;
+}
+
+/* Query fold for the thumbnail scan: the int8 query of R4 (unchanged) and
+ * the factor c2 = (a / 254) / sqrt(D) that maps I_t of R18 to logit units. */
+void ffdo_fold_query_tr(int D, const uint16_t *q_head, const uint16_t *scale_block,
+                        int8_t *qi, float *c_out) {
+  float c127;
+  ffdo_fold_query(D, q_head, scale_block, qi, &c127);
+  float a = 0.0f;
+  for (int c = 0; c < D; ++c) {
+    float ap = fabsf(bf16_to_float(q_head[c]) * bf16_to_float(scale_block[c]));
+    if (ap > a) a = ap;
+  }
+  *c_out = a == 0.0f ? 0.0f : (a / 254.0f) * inv_sqrt_dim(D);
+}
+
+/* Tentative block scores from the thumbnails (R3, R18); layout as
+ * ffdo_block_scores. */
+int ffdo_block_scores_tr(int B, int Hq, int Hkv, int cap, int D, int T,
+                         const uint16_t *q, const uint8_t *thumb, const uint16_t *scales,
+                         const int32_t *lengths, float *scores) {
+  if (check_shape(B, Hq, Hkv, cap, D, T) != FFDO_OK) return FFDO_BAD_ARG;
+  int G = Hq / Hkv, nblk = cap / T;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 0 || lengths[b] > cap) return FFDO_BAD_LENGTH;
+  for (int b = 0; b < B; ++b) {
+    int len = lengths[b];
+    int nb = (len + T - 1) / T;
+    for (int h = 0; h < Hq; ++h) {
+      int g = h / G;
+      size_t row = (size_t)b * Hkv + g;
+      const uint16_t *qh = q + ((size_t)b * Hq + h) * D;
+      const uint8_t *trow = thumb + row * (size_t)cap * (D / 4);
+      const uint16_t *srow = scales + row * (size_t)nblk * D;
+      float *out = scores + ((size_t)b * Hq + h) * nblk;
+      for (int j = 0; j < nblk; ++j) out[j] = -INFINITY;
+      for (int j = 0; j < nb; ++j) {
+        int8_t qi[128];
+        float cj;
+        ffdo_fold_query_tr(D, qh, srow + (size_t)j * D, qi, &cj);
+        int t_end = (j + 1) * T < len ? (j + 1) * T : len;
+        int64_t best = INT64_MIN;
+        for (int t = j * T; t < t_end; ++t) {
+          const uint8_t *tr = trow + (size_t)t * (D / 4);
+          int64_t dot = 0;
+          for (int c = 0; c < D; ++c) dot += (int64_t)qi[c] * (2 * thumb_code(tr, c) - 3);
+          if (dot > best) best = dot;
+        }
+        out[j] = (float)best * cj;
+      }
+    }
+  }
+  return FFDO_OK;
+}
+
+/* The computer's keys: k_hat [B][Hkv][cap][D] (fp64) for t < length, 0 past it. */
+int ffdo_reconstruct_keys_tr(int B, int Hkv, int cap, int D, int T, const uint8_t *thumb,
+                             const uint8_t *resid, const uint16_t *scales,
+                             const int32_t *lengths, double *k_hat) {
+  if (check_shape(B, Hkv, Hkv, cap, D, T) != FFDO_OK) return FFDO_BAD_ARG;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 0 || lengths[b] > cap) return FFDO_BAD_LENGTH;
+  key_source ks = {NULL, thumb, resid, scales};
+  for (int b = 0; b < B; ++b)
+    for (int g = 0; g < Hkv; ++g) {
+      size_t row = (size_t)b * Hkv + g;
+      for (int t = 0; t < cap; ++t)
+        for (int c = 0; c < D; ++c)
+          k_hat[(row * (size_t)cap + (size_t)t) * D + c] =
+              t < lengths[b] ? key_value(&ks, row, cap, D, T, t, c) : 0.0;
+    }
+  return FFDO_OK;
+}
+
+/* fp64 attention over the selected blocks with the reconstructed keys. */
+int ffdo_attend_tr(int B, int Hq, int Hkv, int cap, int D, int T, const uint16_t *q,
+                   const uint8_t *thumb, const uint8_t *resid, const uint16_t *scales,
+                   const uint16_t *v, const int32_t *lengths, const uint32_t *mask,
+                   double *out, double *lse) {
+  key_source ks = {NULL, thumb, resid, scales};
+  return attend_impl(B, Hq, Hkv, cap, D, T, q, &ks, v, lengths, mask, out, lse);
+}
+
+/* The whole step on the thumbnail + residual format: thumbnail scores ->
+ * Top-delta (running max, or the pseudo-max of R15 when pseudo_max != 0) ->
+ * attention with reconstructed keys.  delta = +INF selects every valid block. */
+int ffdo_decode_tr(int B, int Hq, int Hkv, int cap, int D, int T, int S,
+                   const uint16_t *q, const uint16_t *v, const uint8_t *thumb,
+                   const uint8_t *resid, const uint16_t *scales, const int32_t *lengths,
+                   float delta, int pseudo_max, double *out, uint32_t *mask, float *scores) {
+  int rc = check_shape(B, Hq, Hkv, cap, D, T);
+  if (rc != FFDO_OK) return rc;
+  if (S <= 0 || !(delta >= 0.0f)) return FFDO_BAD_ARG;
+  int nblk = cap / T;
+  float *own = NULL;
+  if (!scores) {
+    own = (float *)malloc(sizeof(float) * (size_t)B * Hq * (nblk > 0 ? nblk : 1));
+    if (!own) return FFDO_BAD_ARG;
+    scores = own;
+  }
+  if (isinf(delta)) {
+    for (size_t i = 0; i < (size_t)B * Hq * nblk; ++i) scores[i] = 0.0f;
+    for (int b = 0; b < B; ++b)
+      if (lengths[b] < 0 || lengths[b] > cap) { free(own); return FFDO_BAD_LENGTH; }
+  } else {
+    rc = ffdo_block_scores_tr(B, Hq, Hkv, cap, D, T, q, thumb, scales, lengths, scores);
+    if (rc != FFDO_OK) { free(own); return rc; }
+  }
+  rc = pseudo_max
+           ? ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask)
+           : ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  if (rc == FFDO_OK)
+    rc = ffdo_attend_tr(B, Hq, Hkv, cap, D, T, q, thumb, resid, scales, v, lengths, mask, out, NULL);
   free(own);
   return rc;
 }
