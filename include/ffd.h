@@ -40,6 +40,13 @@
  *   out      bf16 [B][Hq][D]
  *   mask     u32  [B][Hkv][W]                 bit (j % 32) of word j / 32 set iff
  *            block j was selected for that kv-head; bits >= ceil(len/T) are 0
+ *   thumbnail + residual key format (ffd_quantize_keys_tr, ffd_decode_tr):
+ *   k_thumb  u8   [B][Hkv][cap][D/4]          2-bit codes u in [0, 3]: channel
+ *            16w + i of a token row sits in little-endian 32-bit word w at bit
+ *            2 (i / 2) + 16 (i % 2) (even channels of the group in the low
+ *            half-word, odd channels in the high half-word)
+ *   k_resid  u8   [B][Hkv][cap][D]            8-bit residual e + 128, e in [-127, 127]
+ *   k_scales bf16 [B][Hkv][nblk][D]           per-block-per-channel scales (as above)
  */
 #ifndef FFD_H
 #define FFD_H
@@ -182,6 +189,55 @@ ffd_status ffd_decode_ex(const ffd_shape *shape, const ffd_decode_options *optio
                          void *k_scales, const int32_t *d_lengths, float delta, void *out_bf16,
                          uint32_t *mask, void *workspace, size_t workspace_bytes, void *cuda_stream);
 
+/* ---- The pages' own key format: 2-bit thumbnails + 8-bit residuals ----
+ * gist.science explainer, Methodology 1: the K cache is split into 2-bit
+ * quantised thumbnails, scanned to estimate scores, and 8-bit residuals that
+ * with the thumbnails reconstruct the keys to near-16-bit precision for the
+ * exact computation (Methodology 3, "Fine-Grained Refinement": kept blocks
+ * load residuals and values).  The computer then never reads bf16 K: per
+ * token it reads 32 thumbnail + 128 residual + 256 V bytes instead of 64
+ * int4 + 256 K + 256 V bytes. */
+
+/* Bytes of k_thumb and k_resid for the whole batch (k_scales: ffd_scale_bytes).
+ * 0 for an invalid shape. */
+size_t ffd_thumb_bytes(const ffd_shape *shape);
+size_t ffd_residual_bytes(const ffd_shape *shape);
+
+/* Thumbnail + residual copy of the keys, for the same blocks as
+ * ffd_quantize_keys (block_begin, FFD_LAST_BLOCK).  Per (block, channel) over
+ * the block's valid tokens t:
+ *   amax_c = max_t |k[t][c]|,  s_c = bf16_rne(amax_c / 1.5)   (IEEE fp32 division)
+ *   y = k / s_c,  u = clamp(floor(y) + 2, 0, 3)   (level (u - 1.5) s_c)
+ *   e = clamp(rint_even((y - (u - 1.5)) * 254), -127, 127)   (fp32, one rounding per step)
+ *   s_c == 0 gives u = 2, e = 0; tokens at or past lengths[b] in the last
+ *   block are zero bytes (thumbnail and residual) and do not enter amax.
+ * The computer's key is k_hat = s_c (254 u - 381 + e) / 254, within s_c / 508
+ * of k (a 10-bit grid over the block's range). */
+ffd_status ffd_quantize_keys_tr(const ffd_shape *shape, const void *k_bf16,
+                                const int32_t *d_lengths, int32_t block_begin, void *k_thumb,
+                                void *k_resid, void *k_scales, void *cuda_stream);
+
+/* One fused decode step on the thumbnail + residual format.
+ * Selector (skipped when delta == +INFINITY): the int8 query fold of
+ *   ffd_decode, then I_t = sum_c qi_c (2 u_{t,c} - 3) (exact int; the level of
+ *   code u is (2u - 3) s / 2) and score_j = float(max over valid t of I_t) *
+ *   ((a / 254) * (1 / sqrt(128))); Top-delta and the group union exactly as
+ *   ffd_decode_ex (options->reference).
+ * Computer: every query head of the group attends over the kept blocks' valid
+ *   tokens with the reconstructed keys k_hat (f16 tensor-core products of the
+ *   integer codes z = 254 u - 381 + e with the query folded by s / 254, fp32
+ *   accumulation) and bf16 V; splits merged with log-sum-exp; bf16 output.
+ * options: NULL is rejected; requant_last == 1 first re-quantises each
+ *   sequence's last block from k_bf16 (bit-identical to ffd_quantize_keys_tr
+ *   with FFD_LAST_BLOCK), writing k_thumb, k_resid, k_scales.  k_bf16 is read
+ *   only then and may be NULL when requant_last == 0.
+ * Length handling, workspace and errors as ffd_decode. */
+ffd_status ffd_decode_tr(const ffd_shape *shape, const ffd_decode_options *options,
+                         const void *q_bf16, const void *k_bf16, const void *v_bf16, void *k_thumb,
+                         void *k_resid, void *k_scales, const int32_t *d_lengths, float delta,
+                         void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
+                         void *cuda_stream);
+
 /* Context (sequence) sharding across GPUs.  Each rank holds a contiguous
  * shard of every sequence's cache: rank r holds global tokens
  * [r * cap_local, (r + 1) * cap_local) in a cache of capacity cap_local, with
@@ -205,6 +261,13 @@ ffd_status ffd_decode_partials(const ffd_shape *local_shape, const ffd_decode_op
                                void *k_packed, void *k_scales, const int32_t *d_local_lengths,
                                float delta, void *workspace, size_t workspace_bytes,
                                void *cuda_stream);
+/* ffd_decode_partials on the thumbnail + residual format (arguments as
+ * ffd_decode_tr); the exchange and ffd_merge_partials are unchanged. */
+ffd_status ffd_decode_partials_tr(const ffd_shape *local_shape, const ffd_decode_options *options,
+                                  const void *q_bf16, const void *k_bf16, const void *v_bf16,
+                                  void *k_thumb, void *k_resid, void *k_scales,
+                                  const int32_t *d_local_lengths, float delta, void *workspace,
+                                  size_t workspace_bytes, void *cuda_stream);
 ffd_status ffd_partials_region(const ffd_shape *local_shape, size_t *offset, size_t *bytes);
 ffd_status ffd_merge_partials(const ffd_shape *local_shape, int32_t num_shards, const void *gathered,
                               size_t gathered_bytes, const int32_t *d_global_lengths,

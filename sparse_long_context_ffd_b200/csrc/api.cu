@@ -72,6 +72,22 @@ bool make_kv_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Residuals of the thumbnail format as a 2-D u8 tensor {128 bytes, token
+// rows}; one box {128, kKvBoxRows} is one attention stage's residual tile,
+// 128-byte swizzled like the K/V tiles.
+bool make_resid_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kResidRowBytes), rows > 0 ? rows : 1};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kResidRowBytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kResidRowBytes), static_cast<cuuint32_t>(kKvBoxRows)};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                            box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group, int32_t capacity,
@@ -120,6 +136,16 @@ size_t ffd_packed_bytes(const ffd_shape *s) {
   return static_cast<size_t>(s->batch) * s->num_kv_heads * s->capacity * (kHeadDim / 2);
 }
 
+size_t ffd_thumb_bytes(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->num_kv_heads * s->capacity * kThumbRowBytes;
+}
+
+size_t ffd_residual_bytes(const ffd_shape *s) {
+  if (check_shape(s) != FFD_OK) return 0;
+  return static_cast<size_t>(s->batch) * s->num_kv_heads * s->capacity * kResidRowBytes;
+}
+
 size_t ffd_scale_bytes(const ffd_shape *s) {
   if (check_shape(s) != FFD_OK) return 0;
   return static_cast<size_t>(s->batch) * s->num_kv_heads * (s->capacity / s->block_size) * kHeadDim * 2;
@@ -150,16 +176,23 @@ ffd_status ffd_workspace_init(const ffd_shape *s, void *workspace, size_t worksp
   return FFD_OK;
 }
 
-ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32_t *d_lengths,
-                             int32_t block_begin, void *k_packed, void *k_scales, void *cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+ffd_status quantize_common(const ffd_shape *s, const void *k_bf16, const int32_t *d_lengths,
+                           int32_t block_begin, void *packed, void *resid, void *k_scales, int format,
+                           void *cuda_stream) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (block_begin < FFD_LAST_BLOCK) return FFD_ERR_INVALID_ARG;
   const int nblk = s->capacity / s->block_size;
   if (s->batch == 0 || nblk == 0) return FFD_OK;
-  if (k_bf16 == nullptr || d_lengths == nullptr || k_packed == nullptr || k_scales == nullptr)
+  const bool tr = format == kFormatThumbResid;
+  if (k_bf16 == nullptr || d_lengths == nullptr || packed == nullptr || k_scales == nullptr ||
+      (tr && resid == nullptr))
     return FFD_ERR_INVALID_ARG;
-  if (!aligned16(k_bf16) || !aligned16(k_packed) || !aligned16(k_scales) ||
+  if (!aligned16(k_bf16) || !aligned16(packed) || !aligned16(k_scales) || (tr && !aligned16(resid)) ||
       (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
     return FFD_ERR_INVALID_ARG;
   const int blocks = block_begin < 0 ? 1 : nblk - block_begin;
@@ -167,12 +200,14 @@ ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32
   QuantizeParams p{};
   p.k = static_cast<const uint16_t *>(k_bf16);
   p.lengths = d_lengths;
-  p.packed = static_cast<uint8_t *>(k_packed);
+  p.packed = static_cast<uint8_t *>(packed);
   p.scales = static_cast<uint16_t *>(k_scales);
+  p.resid = tr ? static_cast<uint8_t *>(resid) : nullptr;
   p.batch = s->batch;
   p.num_kv_heads = s->num_kv_heads;
   p.capacity = s->capacity;
   p.block_begin = block_begin;
+  p.format = format;
   const dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(s->num_kv_heads),
                   static_cast<unsigned>(s->batch));
   if (launch_quantize(p, s->block_size, grid, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
@@ -180,11 +215,37 @@ ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32
   return FFD_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+ffd_status ffd_quantize_keys(const ffd_shape *s, const void *k_bf16, const int32_t *d_lengths,
+                             int32_t block_begin, void *k_packed, void *k_scales, void *cuda_stream) {
+  return quantize_common(s, k_bf16, d_lengths, block_begin, k_packed, nullptr, k_scales, kFormatInt4,
+                         cuda_stream);
+}
+
+ffd_status ffd_quantize_keys_tr(const ffd_shape *s, const void *k_bf16, const int32_t *d_lengths,
+                                int32_t block_begin, void *k_thumb, void *k_resid, void *k_scales,
+                                void *cuda_stream) {
+  return quantize_common(s, k_bf16, d_lengths, block_begin, k_thumb, k_resid, k_scales, kFormatThumbResid,
+                         cuda_stream);
+}
+
 namespace {
 
-// Shared body of ffd_decode and ffd_decode_step.
-ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
-                         const void *v_bf16, const void *k_packed, const void *k_scales,
+// Where the keys come from: the int4 scan copy beside the bf16 cache, or the
+// thumbnail + residual pair (bf16 K then read only by the re-quantisation).
+struct KeyBuffers {
+  int format;
+  const void *k;       // bf16 K cache
+  const void *packed;  // int4 codes or thumbnails
+  const void *resid;   // residuals (thumbnail format)
+  const void *scales;
+};
+
+// Shared body of every decode entry point.
+ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffers &kb, const void *v_bf16,
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
                          int32_t reference, bool partials_only = false) {
@@ -201,30 +262,37 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
   if (std::isnan(delta) || delta < 0.0f) return FFD_ERR_INVALID_ARG;
   if (s->batch == 0) return FFD_OK;
   const bool dense = std::isinf(delta);
+  const bool tr = kb.format == kFormatThumbResid;
   const int group = s->num_q_heads / s->num_kv_heads;
   const WorkspaceLayout L =
       workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks);
   if (workspace == nullptr || workspace_bytes < L.total) return FFD_ERR_WORKSPACE;
-  if (q_bf16 == nullptr || k_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
+  if (q_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
       (!partials_only && (out_bf16 == nullptr || mask == nullptr)))
     return FFD_ERR_INVALID_ARG;
-  const bool need_packed = requant || !dense;
-  if (need_packed && (k_packed == nullptr || k_scales == nullptr)) return FFD_ERR_INVALID_ARG;
-  if (!aligned16(q_bf16) || !aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
+  // bf16 K: the int4 format's computer reads it; both formats re-quantise from it
+  const bool need_k = !tr || requant;
+  // scan copy: needed by the selector and written by the re-quantisation; the
+  // thumbnail format's computer always reads thumbnails, residuals and scales
+  const bool need_packed = tr || requant || !dense;
+  if (need_k && kb.k == nullptr) return FFD_ERR_INVALID_ARG;
+  if (need_packed && (kb.packed == nullptr || kb.scales == nullptr)) return FFD_ERR_INVALID_ARG;
+  if (tr && kb.resid == nullptr) return FFD_ERR_INVALID_ARG;
+  if (!aligned16(q_bf16) || !aligned16(kb.k) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
       !aligned16(mask) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
-    return FFD_ERR_INVALID_ARG;  // (null out/mask pass: aligned16(nullptr) holds)
-  if (need_packed && (!aligned16(k_packed) || !aligned16(k_scales))) return FFD_ERR_INVALID_ARG;
+    return FFD_ERR_INVALID_ARG;  // (null pointers pass: aligned16(nullptr) holds)
+  if (!aligned16(kb.packed) || !aligned16(kb.scales) || !aligned16(kb.resid)) return FFD_ERR_INVALID_ARG;
 
   const uint64_t rows = static_cast<uint64_t>(s->batch) * s->num_kv_heads * s->capacity;
   CUtensorMap tmap_k, tmap_v;
-  if (!make_kv_tensor_map(&tmap_k, k_bf16, rows) || !make_kv_tensor_map(&tmap_v, v_bf16, rows))
-    return FFD_ERR_CUDA;
+  const bool kmap_ok = tr ? make_resid_tensor_map(&tmap_k, kb.resid, rows) : make_kv_tensor_map(&tmap_k, kb.k, rows);
+  if (!kmap_ok || !make_kv_tensor_map(&tmap_v, v_bf16, rows)) return FFD_ERR_CUDA;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   DecodeParams p{};
   p.q = static_cast<const uint16_t *>(q_bf16);
-  p.packed = static_cast<const uint8_t *>(k_packed);
-  p.scales = static_cast<const uint16_t *>(k_scales);
+  p.packed = static_cast<const uint8_t *>(kb.packed);
+  p.scales = static_cast<const uint16_t *>(kb.scales);
   p.lengths = d_lengths;
   p.out = static_cast<uint16_t *>(out_bf16);
   p.mask = mask;
@@ -244,17 +312,30 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const void *k_b
   p.requant_last = requant ? 1 : 0;
   p.reference = reference;
   p.partials_only = partials_only ? 1 : 0;
-  p.k = static_cast<const uint16_t *>(k_bf16);
-  p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(k_packed)) : nullptr;
-  p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(k_scales)) : nullptr;
+  p.k = static_cast<const uint16_t *>(kb.k);
+  p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(kb.packed)) : nullptr;
+  p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(kb.scales)) : nullptr;
+  p.resid_out = requant && tr ? static_cast<uint8_t *>(const_cast<void *>(kb.resid)) : nullptr;
 
   const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
                   static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
-  const size_t smem = decode_smem_bytes(s->block_size, group, s->split_blocks);
-  if (launch_decode(p, tmap_k, tmap_v, s->block_size, group, grid, smem,
+  const size_t smem = decode_smem_bytes(s->block_size, group, s->split_blocks, kb.format);
+  if (launch_decode(p, tmap_k, tmap_v, s->block_size, group, kb.format, grid, smem,
                     static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
     return FFD_ERR_CUDA;
   return FFD_OK;
+}
+
+KeyBuffers int4_keys(const void *k, const void *packed, const void *scales) {
+  return KeyBuffers{kFormatInt4, k, packed, nullptr, scales};
+}
+
+KeyBuffers tr_keys(const void *k, const void *thumb, const void *resid, const void *scales) {
+  return KeyBuffers{kFormatThumbResid, k, thumb, resid, scales};
+}
+
+bool options_ok(const ffd_decode_options *opt) {
+  return opt != nullptr && (opt->requant_last == 0 || opt->requant_last == 1);
 }
 
 }  // namespace
@@ -263,7 +344,7 @@ ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16
                       const void *k_packed, const void *k_scales, const int32_t *d_lengths, float delta,
                       void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
                       void *cuda_stream) {
-  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, false, FFD_REFERENCE_RUNNING_MAX);
 }
 
@@ -271,7 +352,7 @@ ffd_status ffd_decode_step(const ffd_shape *s, const void *q_bf16, const void *k
                            const void *v_bf16, void *k_packed, void *k_scales,
                            const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                            void *workspace, size_t workspace_bytes, void *cuda_stream) {
-  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, true, FFD_REFERENCE_RUNNING_MAX);
 }
 
@@ -279,10 +360,20 @@ ffd_status ffd_decode_partials(const ffd_shape *s, const ffd_decode_options *opt
                                const void *k_bf16, const void *v_bf16, void *k_packed, void *k_scales,
                                const int32_t *d_local_lengths, float delta, void *workspace,
                                size_t workspace_bytes, void *cuda_stream) {
-  if (opt == nullptr || (opt->requant_last != 0 && opt->requant_last != 1)) return FFD_ERR_INVALID_ARG;
-  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_local_lengths, delta, nullptr,
-                       nullptr, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
+  if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_local_lengths, delta,
+                       nullptr, nullptr, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
                        opt->reference, true);
+}
+
+ffd_status ffd_decode_partials_tr(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,
+                                  const void *k_bf16, const void *v_bf16, void *k_thumb, void *k_resid,
+                                  void *k_scales, const int32_t *d_local_lengths, float delta,
+                                  void *workspace, size_t workspace_bytes, void *cuda_stream) {
+  if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, tr_keys(k_bf16, k_thumb, k_resid, k_scales), v_bf16, d_local_lengths,
+                       delta, nullptr, nullptr, workspace, workspace_bytes, cuda_stream,
+                       opt->requant_last == 1, opt->reference, true);
 }
 
 ffd_status ffd_partials_region(const ffd_shape *s, size_t *offset, size_t *bytes) {
@@ -340,10 +431,19 @@ ffd_status ffd_decode_ex(const ffd_shape *s, const ffd_decode_options *opt, cons
                          const void *k_bf16, const void *v_bf16, void *k_packed, void *k_scales,
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream) {
-  if (opt == nullptr) return FFD_ERR_INVALID_ARG;
-  if (opt->requant_last != 0 && opt->requant_last != 1) return FFD_ERR_INVALID_ARG;
-  return decode_common(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
+  if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
+                       opt->reference);
+}
+
+ffd_status ffd_decode_tr(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,
+                         const void *k_bf16, const void *v_bf16, void *k_thumb, void *k_resid,
+                         void *k_scales, const int32_t *d_lengths, float delta, void *out_bf16,
+                         uint32_t *mask, void *workspace, size_t workspace_bytes, void *cuda_stream) {
+  if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
+  return decode_common(s, q_bf16, tr_keys(k_bf16, k_thumb, k_resid, k_scales), v_bf16, d_lengths, delta,
+                       out_bf16, mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
                        opt->reference);
 }
 

@@ -28,6 +28,7 @@
 // partial, and the last CTA to finish for (b, g) merges all splits and writes
 // the bf16 output rows and the mask row.  No CTA ever waits for another.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <atomic>
 #include <climits>
@@ -52,29 +53,49 @@ constexpr int kThreads = (kAttnWarps + 2) * 32;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kKvTok = kKvBoxRows;                  // tokens per attention stage
 constexpr int kKvHalfBytes = kKvTok * 128;          // one 64-channel half of K or V
-constexpr int kKvStageBytes = 4 * kKvHalfBytes;     // K lo, K hi, V lo, V hi: 16 KiB
-constexpr int kKvStagesN = 5;
-constexpr int kKvRingBytes = kKvStagesN * kKvStageBytes;
 constexpr int kMergeBytes = kAttnWarps * (8 + 8 + 8 * kHeadDim) * 4;
 
-template <int T>
+// One attention stage (kKvTok tokens of one kept block) per key format.
+template <int F>
+struct KvGeom;
+template <>
+struct KvGeom<kFormatInt4> {  // K lo, K hi, V lo, V hi (bf16, 128-byte swizzle): 16 KiB
+  static constexpr int kVOffset = 2 * kKvHalfBytes;
+  static constexpr int kTx = 4 * kKvHalfBytes;
+  static constexpr int kStageBytes = kTx;
+  static constexpr int kStages = 5;
+};
+template <>
+struct KvGeom<kFormatThumbResid> {
+  // residual rows (128 B, 128-byte swizzle) | V lo | V hi | thumbnail rows | scale row
+  static constexpr int kVOffset = kKvTok * kResidRowBytes;
+  static constexpr int kThumbOffset = kVOffset + 2 * kKvHalfBytes;
+  static constexpr int kScaleOffset = kThumbOffset + kKvTok * kThumbRowBytes;
+  static constexpr int kTx = kScaleOffset + kScaleRowBytes;
+  static constexpr int kStageBytes = (kTx + 1023) / 1024 * 1024;  // swizzled tiles stay 1 KiB aligned
+  static constexpr int kStages = 6;
+};
+
+template <int T, int F>
 struct ScanGeom {
-  static constexpr int kStageBytes = T * kPackedRowBytes + kScaleRowBytes;
-  static constexpr int kStages = T == 64 ? 4 : 2;
+  static constexpr int kRowBytes = F == kFormatThumbResid ? kThumbRowBytes : kPackedRowBytes;
+  static constexpr int kStageBytes = T * kRowBytes + kScaleRowBytes;
+  static constexpr int kStages = (F == kFormatThumbResid ? 2 : 1) * (T == 64 ? 4 : 2);
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
 };
 
-template <int T>
+template <int T, int F>
 struct SmemLayout {
+  static constexpr int NKV = KvGeom<F>::kStages;
   static constexpr int kKvRing = 0;
-  static constexpr int kScanRing = kKvRingBytes;
-  static constexpr int kBars = kScanRing + ScanGeom<T>::kRingBytes;
-  static constexpr int kNumBars = 2 * ScanGeom<T>::kStages + 2 * kKvStagesN;
-  static constexpr int kMeta = kBars + 8 * kNumBars;     // int [kKvStagesN] token offsets
-  static constexpr int kSeq = kMeta + 4 * kKvStagesN;    // int [kKvStagesN] item indices
-  static constexpr int kCtrl = kSeq + 4 * kKvStagesN;    // qcount, sel_done, is_last, abort
-  static constexpr int kKeep = kCtrl + 16;               // u32 [split_words]
+  static constexpr int kScanRing = NKV * KvGeom<F>::kStageBytes;
+  static constexpr int kBars = kScanRing + ScanGeom<T, F>::kRingBytes;
+  static constexpr int kNumBars = 2 * ScanGeom<T, F>::kStages + 2 * NKV;
+  static constexpr int kMeta = kBars + 8 * kNumBars;  // int [NKV] token offsets
+  static constexpr int kSeq = kMeta + 4 * NKV;        // int [NKV] item indices
+  static constexpr int kCtrl = kSeq + 4 * NKV;        // qcount, sel_done, is_last, abort
+  static constexpr int kKeep = kCtrl + 16;            // u32 [split_words]
   // queue of kept block indices (u16 [split_blocks]) follows keep bits
 };
 
@@ -85,6 +106,23 @@ __device__ __forceinline__ int clamp127(int x) { return min(127, max(-127, x)); 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Reconstructed key codes z = 254 u - 381 + e of two channels as an f16 pair.
+// `w_shifted` holds the two 2-bit codes at bits 0 and 16; `resid_word` the two
+// residual bytes (e + 128) at byte positions picked by `sel` (0x4140: bytes 0
+// and 1, 0x4342: bytes 2 and 3).  The byte permute puts 0x64 above each byte,
+// so a lane reads as the f16 1024 + (e + 128) + 254 u = z + 1533 exactly (all
+// below 2048); one f16x2 subtraction of 1533 (0x65FD) leaves z exactly.
+__device__ __forceinline__ uint32_t key_pair(uint32_t w_shifted, uint32_t resid_word, uint32_t sel) {
+  const uint32_t u = w_shifted & 0x00030003u;
+  const uint32_t e = __byte_perm(resid_word, 0x64646464u, sel);
+  return sub_f16x2(u * 254u + e, 0x65FD65FDu);
 }
 
 __device__ __forceinline__ void raise_timeout(const DecodeParams &p, volatile int *ctrl) {
@@ -216,13 +254,117 @@ __device__ __forceinline__ void scan_block(const uint8_t *tile, const uint16_t *
   score1 = __fmul_rn(__int2float_rn(best1 - 8 * sq1), c1);
 }
 
+// Selector for one block of 2-bit thumbnails (same contract as scan_block).
+// The fold is the int4 one; the thumbnail level of code u is (2u - 3) s / 2,
+// so I_t = sum_c qi_c (2 u_c - 3) = 2 sum_c qi_c u_c - 3 sum_c qi_c and the
+// score is float(max_t I_t) * (a / 254) / sqrt(D).
+//
+// Lane (gid, t4) again owns channels 32*t4 .. 32*t4 + 31 = thumbnail words
+// 2*t4 and 2*t4 + 1 of a token row.  (w >> 2k) & 0x03030303 puts channels
+// 16w' + {2k, 8+2k, 2k+1, 9+2k} (w' the word's group) in bytes 0..3, so
+// k-step k takes a0 from word 2*t4 and a2 from word 2*t4 + 1, and the int8
+// query is packed in the same channel order.
 template <int T, int G>
+__device__ __forceinline__ void scan_block_tr(const uint8_t *tile, const uint16_t *scl,
+                                              const uint32_t (&qreg)[16], int valid_rows, int lane,
+                                              float &score0, float &score1) {
+  const int gid = lane >> 2, t4 = lane & 3;
+  float pc[32];
+  float a = 0.0f;
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(scl) + 4 * t4;
+#pragma unroll
+  for (int w4 = 0; w4 < 4; ++w4) {
+    const uint4 sv = s4[w4];
+    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int k = 8 * w4 + 2 * e;
+      const uint32_t qw = qreg[k >> 1];
+      pc[k] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
+      pc[k + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
+      a = fmaxf(a, fmaxf(fabsf(pc[k]), fabsf(pc[k + 1])));
+    }
+  }
+  a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
+
+  uint32_t bq[4][2];
+  int sumq = 0;
+  float cf = 0.0f;
+  if (gid < G && a > 0.0f) {
+    const float inv = __fdiv_rn(127.0f, a);
+    int qi[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      qi[c] = clamp127(__float2int_rn(__fmul_rn(pc[c], inv)));
+      sumq += qi[c];
+    }
+    // k-step k, half h (a0: word 2*t4, a2: word 2*t4 + 1): local channels
+    // 16h + {2k, 8+2k, 2k+1, 9+2k} in bytes 0..3
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c0 = 16 * h + 2 * k;
+        bq[k][h] = (static_cast<uint32_t>(qi[c0]) & 0xFFu) | ((static_cast<uint32_t>(qi[c0 + 8]) & 0xFFu) << 8) |
+                   ((static_cast<uint32_t>(qi[c0 + 1]) & 0xFFu) << 16) |
+                   ((static_cast<uint32_t>(qi[c0 + 9]) & 0xFFu) << 24);
+      }
+    }
+    cf = __fmul_rn(__fdiv_rn(a, 254.0f), kRsqrtD);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) bq[k][0] = bq[k][1] = 0u;
+  }
+  sumq += __shfl_xor_sync(kFull, sumq, 1);
+  sumq += __shfl_xor_sync(kFull, sumq, 2);
+
+  int best0 = INT_MIN, best1 = INT_MIN;  // max_t sum_c qi_c u_c, heads 2*t4, 2*t4 + 1
+#pragma unroll
+  for (int mt = 0; mt < T / 16; ++mt) {
+    const int r0 = 16 * mt + gid, r1 = r0 + 8;
+    const uint2 u0 = *reinterpret_cast<const uint2 *>(tile + r0 * kThumbRowBytes + 8 * t4);
+    const uint2 u1 = *reinterpret_cast<const uint2 *>(tile + r1 * kThumbRowBytes + 8 * t4);
+    int acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mma_u8s8_16x8x32(acc, (u0.x >> (2 * k)) & 0x03030303u, (u1.x >> (2 * k)) & 0x03030303u,
+                       (u0.y >> (2 * k)) & 0x03030303u, (u1.y >> (2 * k)) & 0x03030303u, bq[k][0],
+                       bq[k][1]);
+    }
+    if (r0 < valid_rows) {
+      best0 = max(best0, acc[0]);
+      best1 = max(best1, acc[1]);
+    }
+    if (r1 < valid_rows) {
+      best0 = max(best0, acc[2]);
+      best1 = max(best1, acc[3]);
+    }
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    best0 = max(best0, __shfl_xor_sync(kFull, best0, off));
+    best1 = max(best1, __shfl_xor_sync(kFull, best1, off));
+  }
+  const int h0 = 2 * t4, h1 = 2 * t4 + 1;
+  const int sq0 = __shfl_sync(kFull, sumq, h0 << 2);
+  const int sq1 = __shfl_sync(kFull, sumq, h1 << 2);
+  const float c0 = __shfl_sync(kFull, cf, h0 << 2);
+  const float c1 = __shfl_sync(kFull, cf, h1 << 2);
+  score0 = __fmul_rn(__int2float_rn(2 * best0 - 3 * sq0), c0);
+  score1 = __fmul_rn(__int2float_rn(2 * best1 - 3 * sq1), c1);
+}
+
+template <int T, int G, int F>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
-  using SG = ScanGeom<T>;
-  using SL = SmemLayout<T>;
+  using SG = ScanGeom<T, F>;
+  using SL = SmemLayout<T, F>;
+  using KG = KvGeom<F>;
+  constexpr bool kTR = F == kFormatThumbResid;
   constexpr int NSA = SG::kStages;
+  constexpr int NKV = KG::kStages;
   constexpr int kSubPerBlock = T / kKvTok;
 
   extern __shared__ uint8_t smem_raw[];
@@ -234,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t *full_a = bars;
   uint64_t *empty_a = full_a + NSA;
   uint64_t *full_b = empty_a + NSA;
-  uint64_t *empty_b = full_b + kKvStagesN;
+  uint64_t *empty_b = full_b + NKV;
   volatile int *meta = reinterpret_cast<volatile int *>(smem + SL::kMeta);
   volatile int *seq = reinterpret_cast<volatile int *>(smem + SL::kSeq);
   volatile int *ctrl = reinterpret_cast<volatile int *>(smem + SL::kCtrl);  // qcount, done, last, abort
@@ -280,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&full_a[s], 1);
       mbar_init(&empty_a[s], 1);
     }
-    for (int s = 0; s < kKvStagesN; ++s) {
+    for (int s = 0; s < NKV; ++s) {
       mbar_init(&full_b[s], 1);
       mbar_init(&empty_b[s], 1);
       seq[s] = -1;
@@ -304,11 +446,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int jl = nb - 1;
       const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
       float *red = reinterpret_cast<float *>(scan_ring);  // idle until the scan starts
-      quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
-                                      p.packed_out + tok0 * kPackedRowBytes,
-                                      p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim,
-                                      red, red + (kAttnThreads / 32) * kHeadDim,
-                                      static_cast<int>(threadIdx.x), 2);
+      uint16_t *scale_row = p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim;
+      if constexpr (kTR)
+        quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                           p.packed_out + tok0 * kThumbRowBytes,
+                                           p.resid_out + tok0 * kResidRowBytes, scale_row, red,
+                                           red + (kAttnThreads / 32) * kHeadDim,
+                                           static_cast<int>(threadIdx.x), 2);
+      else
+        quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                        p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
+                                        red + (kAttnThreads / 32) * kHeadDim,
+                                        static_cast<int>(threadIdx.x), 2);
       fence_proxy_async_global();
     }
     fence_proxy_async_smem();
@@ -318,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ================================================================ producer
   if (warp == kProducerWarp) {
     if (lane != 0) return;
-    const uint8_t *src_p = p.packed + row * p.capacity * kPackedRowBytes;
+    const uint8_t *src_p = p.packed + row * p.capacity * SG::kRowBytes;
     const uint16_t *src_s = p.scales + row * static_cast<size_t>(p.capacity / T) * kHeadDim;
     const int row_tok0 = static_cast<int>(row * p.capacity);
     const int scan_total = dense ? 0 : nref + nbs;
@@ -341,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int jb = scan_block_index(sc_next, nref, nb, j0);
         uint8_t *dst = scan_ring + st * SG::kStageBytes;
         mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
-        bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * kPackedRowBytes, T * kPackedRowBytes,
+        bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * SG::kRowBytes, T * SG::kRowBytes,
                  &full_a[st]);
-        bulk_g2s(dst + T * kPackedRowBytes, src_s + static_cast<size_t>(jb) * kHeadDim,
+        bulk_g2s(dst + T * SG::kRowBytes, src_s + static_cast<size_t>(jb) * kHeadDim,
                  kScaleRowBytes, &full_a[st]);
         ++sc_next;
         progress = true;
@@ -360,16 +509,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           sub = 0;
           continue;
         }
-        const int st = it_next % kKvStagesN;
-        const int use = it_next / kKvStagesN;
+        const int st = it_next % NKV;
+        const int use = it_next / NKV;
         if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
-        uint8_t *dst = kv_ring + st * kKvStageBytes;
+        uint8_t *dst = kv_ring + st * KG::kStageBytes;
         meta[st] = tok;
         seq[st] = it_next;
-        mbar_arrive_expect_tx(&full_b[st], kKvStageBytes);
+        mbar_arrive_expect_tx(&full_b[st], KG::kTx);
         const int y = row_tok0 + tok;
-        tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);                 // K: both halves
-        tma_load_3d(dst + 2 * kKvHalfBytes, &tmap_v, 0, y, 0, &full_b[st]);  // V: both halves
+        if constexpr (kTR) {
+          tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);  // residual rows
+          bulk_g2s(dst + KG::kThumbOffset, src_p + static_cast<size_t>(tok) * kThumbRowBytes,
+                   kKvTok * kThumbRowBytes, &full_b[st]);
+          bulk_g2s(dst + KG::kScaleOffset, src_s + static_cast<size_t>(tok / T) * kHeadDim,
+                   kScaleRowBytes, &full_b[st]);
+        } else {
+          tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);  // K: both halves
+        }
+        tma_load_3d(dst + KG::kVOffset, &tmap_v, 0, y, 0, &full_b[st]);  // V: both halves
         ++it_next;
         ++sub;
         progress = true;
@@ -378,8 +535,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       // end marker per attention warp
       if (sel_done && q_ptr >= avail) {
         while (ends_sent < kAttnWarps) {
-          const int st = it_next % kKvStagesN;
-          const int use = it_next / kKvStagesN;
+          const int st = it_next % NKV;
+          const int use = it_next / NKV;
           if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
           meta[st] = -1;
           seq[st] = it_next;
@@ -405,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     drain_ring(full_a, NSA, sc_next);  // (a skipped entry's phase is completed by its builders)
-    drain_ring(full_b, kKvStagesN, it_next);
+    drain_ring(full_b, NKV, it_next);
     return;
   }
 
@@ -441,8 +598,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int jb = scan_block_index(e, nref, nb, j0);
       const uint8_t *tile = scan_ring + st * SG::kStageBytes;
       float s0, s1;
-      scan_block<T, G>(tile, reinterpret_cast<const uint16_t *>(tile + T * kPackedRowBytes), qreg,
-                       min(T, len - jb * T), lane, s0, s1);
+      const uint16_t *scl = reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes);
+      if constexpr (kTR)
+        scan_block_tr<T, G>(tile, scl, qreg, min(T, len - jb * T), lane, s0, s1);
+      else
+        scan_block<T, G>(tile, scl, qreg, min(T, len - jb * T), lane, s0, s1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_a[st]);
       if (e < nref) {  // reference blocks: the split's running max starts at their max
@@ -483,8 +643,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // ======================================================= attention warps
   const int gid = lane >> 2, t4 = lane & 3;
-  // Q^T as the mma B operand: k-step ks holds channels 16ks + 2*t4 (+1) and
-  // 16ks + 8 + 2*t4 (+1) of head gid.
+  // int4 format -- Q^T as the bf16 mma B operand: k-step ks holds channels
+  // 16ks + 2*t4 (+1) and 16ks + 8 + 2*t4 (+1) of head gid.
+  // thumbnail format -- the bf16 pairs of channels 32*t4 + 2i (+1) of head gid,
+  // folded with each block's scales into f16 per stage.
   uint32_t qb[8][2];
   {
     const uint32_t *qh = reinterpret_cast<const uint32_t *>(
@@ -492,8 +654,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                   kHeadDim);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qb[ks][0] = gid < G ? qh[8 * ks + t4] : 0u;
-      qb[ks][1] = gid < G ? qh[8 * ks + 4 + t4] : 0u;
+      if constexpr (kTR) {
+        qb[ks][0] = gid < G ? qh[16 * t4 + 2 * ks] : 0u;
+        qb[ks][1] = gid < G ? qh[16 * t4 + 2 * ks + 1] : 0u;
+      } else {
+        qb[ks][0] = gid < G ? qh[8 * ks + t4] : 0u;
+        qb[ks][1] = gid < G ? qh[8 * ks + 4 + t4] : 0u;
+      }
     }
   }
   if (local_in_smem) {
@@ -503,10 +670,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int jl = nb - 1;
     uint8_t *tile = scan_ring + 1 * SG::kStageBytes;
     float *red = reinterpret_cast<float *>(kv_ring);
-    quantize_block<T, kAttnThreads>(p.k + (row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T) * kHeadDim,
-                                    min(T, len - jl * T), tile,
-                                    reinterpret_cast<uint16_t *>(tile + T * kPackedRowBytes), red,
-                                    red + (kAttnThreads / 32) * kHeadDim, static_cast<int>(threadIdx.x), 2);
+    const uint16_t *k_rows = p.k + (row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T) * kHeadDim;
+    uint16_t *scale_row = reinterpret_cast<uint16_t *>(tile + T * SG::kRowBytes);
+    if constexpr (kTR)
+      quantize_block_tr<T, kAttnThreads>(k_rows, min(T, len - jl * T), tile, nullptr, scale_row, red,
+                                         red + (kAttnThreads / 32) * kHeadDim,
+                                         static_cast<int>(threadIdx.x), 2);
+    else
+      quantize_block<T, kAttnThreads>(k_rows, min(T, len - jl * T), tile, scale_row, red,
+                                      red + (kAttnThreads / 32) * kHeadDim, static_cast<int>(threadIdx.x), 2);
     fence_proxy_async_smem();  // both regions are later written by async copies
     named_barrier(2, kAttnThreads);
     if (threadIdx.x == 0) mbar_arrive(&full_a[1]);
@@ -530,36 +702,102 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t kv_ring_addr = smem_addr(kv_ring);
 
   for (int it = warp;; it += kAttnWarps) {
-    const int st = it % kKvStagesN;
+    const int st = it % NKV;
     // Items go to the attention warps round-robin, so a warp can reach item
     // `it` before the stage's previous fill (another warp's item) has landed;
     // a parity wait could then match that older phase.  The producer writes
     // `it` into seq[st] only after the previous fill was consumed, so once it
     // is visible the parity below names exactly this fill.
     if (!wait_item_published(seq, st, it) ||
-        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / kKvStagesN) & 1u, kWaitLimitNs)) {
+        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / NKV) & 1u, kWaitLimitNs)) {
       raise_timeout(p, ctrl);
       break;
     }
     const int tok = meta[st];
     if (tok < 0) break;
-    const uint32_t kbase = kv_ring_addr + st * kKvStageBytes;
-    const uint32_t vbase = kbase + 2 * kKvHalfBytes;
+    const uint32_t kbase = kv_ring_addr + st * KG::kStageBytes;
+    const uint32_t vbase = kbase + KG::kVOffset;
 
     // S^T = K Q^T for kKvTok tokens: kKvTok/16 independent accumulator chains
     constexpr int MT = kKvTok / 16;
     float sacc[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.0f;
+    float sc0 = kScaleLog2, sc1 = kScaleLog2;  // logit scale of heads 2*t4, 2*t4 + 1
+    if constexpr (kTR) {
+      // Keys are rebuilt from thumbnail + residual as k_hat = s z / 254 with
+      // the integer z = 254 u - 381 + e (exact in f16).  The block's scales go
+      // into the query instead: q'_c = f16(q_c s_c 2^E / 254), E per head so
+      // that max |q'| is about 2^13 (no f16 overflow or underflow), and the
+      // scores are scaled back by 2^-E in fp32.
+      const uint8_t *stage = kv_ring + st * KG::kStageBytes;
+      const uint4 *s4 = reinterpret_cast<const uint4 *>(stage + KG::kScaleOffset) + 4 * t4;
+      float fq[32];
+      float am = 0.0f;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int chunk = 2 * ks + k_chi;
+      for (int w4 = 0; w4 < 4; ++w4) {
+        const uint4 sv = s4[w4];
+        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * w4 + e;  // channel pair 32*t4 + 2i
+          const uint32_t qw = qb[i >> 1][i & 1];
+          fq[2 * i] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
+          fq[2 * i + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
+          am = fmaxf(am, fmaxf(fabsf(fq[2 * i]), fabsf(fq[2 * i + 1])));
+        }
+      }
+      am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
+      const int ea = static_cast<int>((__float_as_uint(am) >> 23) & 0xFFu);
+      const int E = min(148 - ea, 126);  // am 2^E in [2^21, 2^22)
+      const float mult = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 + E) << 23) * (1.0f / 254.0f);
+      const float uns = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - E) << 23) * kScaleLog2;
+      uint32_t qh[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qh[i] = pack_f16x2(fq[2 * i] * mult, fq[2 * i + 1] * mult);
+      sc0 = __shfl_sync(kFull, uns, (2 * t4) << 2);
+      sc1 = __shfl_sync(kFull, uns, (2 * t4 + 1) << 2);
+      // Lane (gid, t4) supplies channels 32*t4 + 16h + {2k, 2k+1} (a0/a1) and
+      // {2k+8, 2k+9} (a2/a3) at k-step (h, k): thumbnail word 2*t4 + h and
+      // residual chunk 2*t4 + h of rows gid and gid + 8 (both rows = gid mod
+      // 8, so the swizzle XOR is gid).
+      const uint8_t *thumb_s = stage + KG::kThumbOffset;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        const int r = 16 * mt + k_row;
-        uint32_t a[4];
-        ldmatrix_x4(a, kbase + (chunk >> 3) * kKvHalfBytes + r * 128 + (((chunk & 7) ^ r7) << 4));
-        mma_bf16_16x8x16(sacc[mt], a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+        const int r0 = 16 * mt + gid, r1 = r0 + 8;
+        const uint2 w0 = *reinterpret_cast<const uint2 *>(thumb_s + r0 * kThumbRowBytes + 8 * t4);
+        const uint2 w1 = *reinterpret_cast<const uint2 *>(thumb_s + r1 * kThumbRowBytes + 8 * t4);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int chunk = ((2 * t4 + h) ^ gid) << 4;
+          const uint4 e0 = *reinterpret_cast<const uint4 *>(stage + r0 * kResidRowBytes + chunk);
+          const uint4 e1 = *reinterpret_cast<const uint4 *>(stage + r1 * kResidRowBytes + chunk);
+          const uint32_t x0[4] = {e0.x, e0.y, e0.z, e0.w};
+          const uint32_t x1[4] = {e1.x, e1.y, e1.z, e1.w};
+          const uint32_t tw0 = h ? w0.y : w0.x, tw1 = h ? w1.y : w1.x;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t sel = (k & 1) ? 0x4342u : 0x4140u;
+            const uint32_t a0 = key_pair(tw0 >> (2 * k), x0[k >> 1], sel);
+            const uint32_t a1 = key_pair(tw1 >> (2 * k), x1[k >> 1], sel);
+            const uint32_t a2 = key_pair(tw0 >> (2 * k + 8), x0[2 + (k >> 1)], sel);
+            const uint32_t a3 = key_pair(tw1 >> (2 * k + 8), x1[2 + (k >> 1)], sel);
+            mma_f16_16x8x16(sacc[mt], a0, a1, a2, a3, qh[8 * h + k], qh[8 * h + k + 4]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int chunk = 2 * ks + k_chi;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int r = 16 * mt + k_row;
+          uint32_t a[4];
+          ldmatrix_x4(a, kbase + (chunk >> 3) * kKvHalfBytes + r * 128 + (((chunk & 7) ^ r7) << 4));
+          mma_bf16_16x8x16(sacc[mt], a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+        }
       }
     }
     // online softmax (base 2); tokens at or past the length are masked
@@ -568,10 +806,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int mt = 0; mt < MT; ++mt) {
       const int t_lo = tok + 16 * mt + gid;
       const bool v_lo = t_lo < len, v_hi = t_lo + 8 < len;
-      sacc[mt][0] = v_lo ? sacc[mt][0] * kScaleLog2 : -INFINITY;
-      sacc[mt][1] = v_lo ? sacc[mt][1] * kScaleLog2 : -INFINITY;
-      sacc[mt][2] = v_hi ? sacc[mt][2] * kScaleLog2 : -INFINITY;
-      sacc[mt][3] = v_hi ? sacc[mt][3] * kScaleLog2 : -INFINITY;
+      sacc[mt][0] = v_lo ? sacc[mt][0] * sc0 : -INFINITY;
+      sacc[mt][1] = v_lo ? sacc[mt][1] * sc1 : -INFINITY;
+      sacc[mt][2] = v_hi ? sacc[mt][2] * sc0 : -INFINITY;
+      sacc[mt][3] = v_hi ? sacc[mt][3] * sc1 : -INFINITY;
       mx0 = fmaxf(mx0, fmaxf(sacc[mt][0], sacc[mt][2]));
       mx1 = fmaxf(mx1, fmaxf(sacc[mt][1], sacc[mt][3]));
     }
@@ -705,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
   float *stats = reinterpret_cast<float *>(scan_ring);  // [G][2]: M*, L*
   float *wts = stats + 16;                              // [chunk][G]
-  constexpr int kWtsFloats = ScanGeom<T>::kRingBytes / 4 - 16;
+  constexpr int kWtsFloats = SG::kRingBytes / 4 - 16;
   const int chunk = kWtsFloats / G;
   for (int h = warp; h < G; h += kAttnWarps) {
     float m = -INFINITY, l = 0.0f;
@@ -797,10 +1035,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) p.counters[row] = 0u;
 }
 
-template <int T, int G>
-cudaError_t launch_tg(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
-                      size_t smem, cudaStream_t stream) {
-  auto kern = decode_kernel<T, G>;
+template <int T, int F>
+size_t smem_bytes_tf(int split_blocks) {
+  const int split_words = (split_blocks + 31) / 32;
+  return 1024 + SmemLayout<T, F>::kKeep + 4 * static_cast<size_t>((split_words + 3) & ~3) +
+         2 * static_cast<size_t>((split_blocks + 7) & ~7);
+}
+
+template <int T, int G, int F>
+cudaError_t launch_tgf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
+                       size_t smem, cudaStream_t stream) {
+  auto kern = decode_kernel<T, G, F>;
   // Raise the dynamic shared memory cap once per device, to the largest
   // split this build accepts, so later launches (and graph captures) need
   // no attribute call.
@@ -811,7 +1056,7 @@ cudaError_t launch_tg(const DecodeParams &p, const CUtensorMap &tk, const CUtens
   const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
   if (bit == 0 || (configured.load(std::memory_order_acquire) & bit) == 0) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(decode_smem_bytes(T, G, FFD_MAX_SPLIT_BLOCKS)));
+                             static_cast<int>(smem_bytes_tf<T, F>(FFD_MAX_SPLIT_BLOCKS)));
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -819,36 +1064,44 @@ cudaError_t launch_tg(const DecodeParams &p, const CUtensorMap &tk, const CUtens
   return cudaGetLastError();
 }
 
-template <int T>
-cudaError_t launch_t(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int group,
-                     dim3 grid, size_t smem, cudaStream_t stream) {
+template <int T, int F>
+cudaError_t launch_tf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int group,
+                      dim3 grid, size_t smem, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_tg<T, 1>(p, tk, tv, grid, smem, stream);
-    case 2: return launch_tg<T, 2>(p, tk, tv, grid, smem, stream);
-    case 4: return launch_tg<T, 4>(p, tk, tv, grid, smem, stream);
-    case 8: return launch_tg<T, 8>(p, tk, tv, grid, smem, stream);
+    case 1: return launch_tgf<T, 1, F>(p, tk, tv, grid, smem, stream);
+    case 2: return launch_tgf<T, 2, F>(p, tk, tv, grid, smem, stream);
+    case 4: return launch_tgf<T, 4, F>(p, tk, tv, grid, smem, stream);
+    case 8: return launch_tgf<T, 8, F>(p, tk, tv, grid, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int T>
-size_t smem_bytes_t(int split_blocks) {
-  const int split_words = (split_blocks + 31) / 32;
-  return 1024 + SmemLayout<T>::kKeep + 4 * static_cast<size_t>((split_words + 3) & ~3) +
-         2 * static_cast<size_t>((split_blocks + 7) & ~7);
+template <int F>
+cudaError_t launch_f(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int block_size,
+                     int group, dim3 grid, size_t smem, cudaStream_t stream) {
+  if (block_size == 64) return launch_tf<64, F>(p, tk, tv, group, grid, smem, stream);
+  if (block_size == 128) return launch_tf<128, F>(p, tk, tv, group, grid, smem, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-size_t decode_smem_bytes(int block_size, int group, int split_blocks) {
+size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format) {
   (void)group;
-  return block_size == 64 ? smem_bytes_t<64>(split_blocks) : smem_bytes_t<128>(split_blocks);
+  if (format == kFormatThumbResid)
+    return block_size == 64 ? smem_bytes_tf<64, kFormatThumbResid>(split_blocks)
+                            : smem_bytes_tf<128, kFormatThumbResid>(split_blocks);
+  return block_size == 64 ? smem_bytes_tf<64, kFormatInt4>(split_blocks)
+                          : smem_bytes_tf<128, kFormatInt4>(split_blocks);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
-                          int block_size, int group, dim3 grid, size_t smem_bytes, cudaStream_t stream) {
-  if (block_size == 64) return launch_t<64>(p, tmap_k, tmap_v, group, grid, smem_bytes, stream);
-  if (block_size == 128) return launch_t<128>(p, tmap_k, tmap_v, group, grid, smem_bytes, stream);
+                          int block_size, int group, int format, dim3 grid, size_t smem_bytes,
+                          cudaStream_t stream) {
+  if (format == kFormatThumbResid)
+    return launch_f<kFormatThumbResid>(p, tmap_k, tmap_v, block_size, group, grid, smem_bytes, stream);
+  if (format == kFormatInt4)
+    return launch_f<kFormatInt4>(p, tmap_k, tmap_v, block_size, group, grid, smem_bytes, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -12,7 +12,14 @@ namespace ffd {
 
 constexpr int kHeadDim = 128;
 constexpr int kPackedRowBytes = kHeadDim / 2;  // 64 bytes of nibbles per token
+constexpr int kThumbRowBytes = kHeadDim / 4;   // 32 bytes of 2-bit codes per token
+constexpr int kResidRowBytes = kHeadDim;       // 128 residual bytes per token
 constexpr int kScaleRowBytes = kHeadDim * 2;   // 128 bf16 scales per block
+
+// Key formats: the int4 scan copy beside the bf16 cache, or the pages' split
+// of K into 2-bit thumbnails and 8-bit residuals (no bf16 K on the read path).
+constexpr int kFormatInt4 = 0;
+constexpr int kFormatThumbResid = 1;
 
 // Rows of one TMA box of K or V (tokens per attention pipeline stage); a box
 // is 64 channels (128 bytes, the swizzle span) wide.
@@ -25,7 +32,7 @@ constexpr uint32_t kFlagTimeout = 0x2u;
 
 struct DecodeParams {
   const uint16_t *q;       // bf16 [B][Hq][D]
-  const uint8_t *packed;   // [B][Hkv][cap][64]
+  const uint8_t *packed;   // scan copy: int4 [B][Hkv][cap][64] or thumbnails [B][Hkv][cap][32]
   const uint16_t *scales;  // bf16 [B][Hkv][nblk][D]
   const int32_t *lengths;  // [B]
   uint16_t *out;           // bf16 [B][Hq][D]
@@ -45,6 +52,7 @@ struct DecodeParams {
   const uint16_t *k;         // bf16 [B][Hkv][cap][D] (read by the re-quantisation)
   uint8_t *packed_out;       // = packed, written for the last block
   uint16_t *scales_out;      // = scales, written for the last block
+  uint8_t *resid_out;        // thumbnail format: residuals [B][Hkv][cap][128], last block
   // context sharding: write the split partials and bits only (no final merge;
   // out and mask unused)
   int32_t partials_only;
@@ -64,9 +72,10 @@ struct MergeParams {
 struct QuantizeParams {
   const uint16_t *k;
   const int32_t *lengths;
-  uint8_t *packed;
+  uint8_t *packed;  // int4 rows, or thumbnail rows in the thumbnail format
   uint16_t *scales;
-  int32_t batch, num_kv_heads, capacity, block_begin;
+  uint8_t *resid;   // thumbnail format only
+  int32_t batch, num_kv_heads, capacity, block_begin, format;
 };
 
 // Workspace carve-up (byte offsets), identical on host and device.
@@ -78,15 +87,17 @@ struct WorkspaceLayout {
 WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group,
                                  int32_t capacity, int32_t block_size, int32_t split_blocks);
 
-size_t decode_smem_bytes(int block_size, int group, int split_blocks);
+size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format);
 
 size_t merge_smem_bytes(int num_shards, int nsplit_max);
 cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 grid,
                          cudaStream_t stream);
 cudaError_t launch_quantize(const QuantizeParams &p, int block_size, dim3 grid,
                             cudaStream_t stream);
+// tmap_k maps the bf16 K cache (int4 format) or the residuals (thumbnail
+// format); tmap_v the bf16 V cache.
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k,
-                          const CUtensorMap &tmap_v, int block_size, int group, dim3 grid,
-                          size_t smem_bytes, cudaStream_t stream);
+                          const CUtensorMap &tmap_v, int block_size, int group, int format,
+                          dim3 grid, size_t smem_bytes, cudaStream_t stream);
 
 }  // namespace ffd

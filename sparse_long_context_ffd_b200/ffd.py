@@ -34,6 +34,8 @@ EXPORTED = (
     "ffd_workspace_init", "ffd_quantize_keys", "ffd_decode", "ffd_check_device_status",
     "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc", "ffd_decode_step",
     "ffd_decode_ex", "ffd_decode_partials", "ffd_partials_region", "ffd_merge_partials",
+    "ffd_thumb_bytes", "ffd_residual_bytes", "ffd_quantize_keys_tr", "ffd_decode_tr",
+    "ffd_decode_partials_tr",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -87,13 +89,21 @@ def load_library() -> ctypes.CDLL:
             sp = ctypes.POINTER(Shape)
             p, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
             for name in ("ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words",
-                         "ffd_decode_workspace_bytes"):
+                         "ffd_decode_workspace_bytes", "ffd_thumb_bytes", "ffd_residual_bytes"):
                 getattr(lib, name).argtypes = [sp]
                 getattr(lib, name).restype = sz
             lib.ffd_workspace_init.argtypes = [sp, p, sz, p]
             lib.ffd_workspace_init.restype = st
             lib.ffd_quantize_keys.argtypes = [sp, p, p, ctypes.c_int32, p, p, p]
             lib.ffd_quantize_keys.restype = st
+            lib.ffd_quantize_keys_tr.argtypes = [sp, p, p, ctypes.c_int32, p, p, p, p]
+            lib.ffd_quantize_keys_tr.restype = st
+            lib.ffd_decode_tr.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p, p,
+                                          ctypes.c_float, p, p, p, sz, p]
+            lib.ffd_decode_tr.restype = st
+            lib.ffd_decode_partials_tr.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p,
+                                                   p, p, p, ctypes.c_float, p, sz, p]
+            lib.ffd_decode_partials_tr.restype = st
             lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode.restype = st
             lib.ffd_decode_ex.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p,
@@ -161,6 +171,14 @@ def scale_bytes(shape: Shape) -> int:
     return int(load_library().ffd_scale_bytes(ctypes.byref(shape)))
 
 
+def thumb_bytes(shape: Shape) -> int:
+    return int(load_library().ffd_thumb_bytes(ctypes.byref(shape)))
+
+
+def residual_bytes(shape: Shape) -> int:
+    return int(load_library().ffd_residual_bytes(ctypes.byref(shape)))
+
+
 def mask_words(shape: Shape) -> int:
     return int(load_library().ffd_mask_words(ctypes.byref(shape)))
 
@@ -180,6 +198,42 @@ def quantize_keys(shape: Shape, k, lengths, block_begin: int, k_packed, k_scales
     _check(load_library().ffd_quantize_keys(ctypes.byref(shape), _ptr(k), _ptr(lengths),
                                             int(block_begin), _ptr(k_packed), _ptr(k_scales),
                                             _stream(stream)), "ffd_quantize_keys")
+
+
+def quantize_keys_tr(shape: Shape, k, lengths, block_begin: int, k_thumb, k_resid, k_scales,
+                     stream=None) -> None:
+    """2-bit thumbnails + 8-bit residuals (+ bf16 scales) of the keys."""
+    _check(load_library().ffd_quantize_keys_tr(ctypes.byref(shape), _ptr(k), _ptr(lengths),
+                                               int(block_begin), _ptr(k_thumb), _ptr(k_resid),
+                                               _ptr(k_scales), _stream(stream)),
+           "ffd_quantize_keys_tr")
+
+
+def decode_tr(shape: Shape, q, k, v, k_thumb, k_resid, k_scales, lengths, delta: float, out,
+              mask, workspace, reference: int = FFD_REFERENCE_RUNNING_MAX,
+              requant_last: bool = False, stream=None) -> None:
+    """Decode step on the thumbnail + residual key format (k is read only when
+    requant_last re-quantises the last block; it may be None otherwise)."""
+    opts = DecodeOptions(int(reference), 1 if requant_last else 0)
+    _check(load_library().ffd_decode_tr(ctypes.byref(shape), ctypes.byref(opts), _ptr(q), _ptr(k),
+                                         _ptr(v), _ptr(k_thumb), _ptr(k_resid), _ptr(k_scales),
+                                         _ptr(lengths), float(delta), _ptr(out), _ptr(mask),
+                                         _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)), "ffd_decode_tr")
+
+
+def decode_partials_tr(local_shape: Shape, q, k, v, k_thumb, k_resid, k_scales, local_lengths,
+                       delta: float, workspace, requant_last: bool = False, stream=None) -> None:
+    """Context shard on the thumbnail + residual format (see decode_partials)."""
+    opts = DecodeOptions(FFD_REFERENCE_RUNNING_MAX, 1 if requant_last else 0)
+    _check(load_library().ffd_decode_partials_tr(ctypes.byref(local_shape), ctypes.byref(opts),
+                                                  _ptr(q), _ptr(k), _ptr(v), _ptr(k_thumb),
+                                                  _ptr(k_resid), _ptr(k_scales),
+                                                  _ptr(local_lengths), float(delta),
+                                                  _ptr(workspace),
+                                                  workspace.numel() * workspace.element_size(),
+                                                  _stream(stream)), "ffd_decode_partials_tr")
 
 
 def decode(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out, mask,
@@ -286,3 +340,15 @@ class DecodeBuffers:
         self.workspace = torch.empty((max(ws, 256) + 15) // 16 * 16, dtype=torch.uint8,
                                      device=device)
         workspace_init(shape, self.workspace)
+
+
+class ThumbResidBuffers(DecodeBuffers):
+    """DecodeBuffers plus the thumbnail + residual key copy (k_packed unused)."""
+
+    def __init__(self, shape: Shape, device="cuda"):
+        import torch
+        super().__init__(shape, device)
+        B, Hkv, cap, D = shape.batch, shape.num_kv_heads, shape.capacity, shape.head_dim
+        self.k_packed = None
+        self.k_thumb = torch.empty((B, Hkv, cap, D // 4), dtype=torch.uint8, device=device)
+        self.k_resid = torch.empty((B, Hkv, cap, D), dtype=torch.uint8, device=device)

@@ -56,6 +56,8 @@ def test_buffer_sizes(B, Hq, Hkv, cap, T, S):
     assert ffd.packed_bytes(s) == B * Hkv * cap * 64
     assert ffd.scale_bytes(s) == B * Hkv * (cap // T) * 128 * 2
     assert ffd.mask_words(s) == B * Hkv * math.ceil(cap // T / 32)
+    assert ffd.thumb_bytes(s) == B * Hkv * cap * 32
+    assert ffd.residual_bytes(s) == B * Hkv * cap * 128
     nsplit = math.ceil(cap // T / S)
     partials = B * Hkv * nsplit * (Hq // Hkv) * 132 * 4
     ws = ffd.decode_workspace_bytes(s)
@@ -123,6 +125,45 @@ def test_bad_arguments_rejected_on_host():
                                  a, ws, None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_decode_ex(ctypes.byref(s), None, a, a, a, a, a, a, 1.0, a, a, a, ws,
                              None) == ffd.FFD_ERR_INVALID_ARG
+
+
+def test_thumb_resid_arguments_rejected_on_host():
+    lib = ffd.load_library()
+    s = ffd.make_shape(2, 16, 4, 4096, 64, 16)
+    ws = ffd.decode_workspace_bytes(s)
+    a = 1 << 20
+    run = ffd.DecodeOptions(0, 0)
+    step = ffd.DecodeOptions(0, 1)
+
+    def dec(opt=run, q=a, k=a, v=a, th=a, re=a, sc=a, ln=a, delta=1.0, out=a, mask=a, w=a, wb=ws):
+        o = None if opt is None else ctypes.byref(opt)
+        return lib.ffd_decode_tr(ctypes.byref(s), o, q, k, v, th, re, sc, ln, delta, out, mask, w,
+                                 wb, None)
+
+    assert dec(opt=None) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(opt=ffd.DecodeOptions(0, 3)) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(delta=float("nan")) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(wb=ws - 1) == ffd.FFD_ERR_WORKSPACE
+    for name in ("q", "v", "th", "re", "sc", "ln", "out", "mask"):
+        assert dec(**{name: None}) == ffd.FFD_ERR_INVALID_ARG, name
+        assert dec(**{name: a + 2}) == ffd.FFD_ERR_INVALID_ARG, name
+    # the computer reconstructs keys from thumbnails and residuals, so they are
+    # needed in dense mode too; bf16 K only when the last block is re-quantised
+    assert dec(th=None, delta=float("inf")) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(opt=step, k=None) == ffd.FFD_ERR_INVALID_ARG
+    assert dec(opt=step, k=a + 8) == ffd.FFD_ERR_INVALID_ARG
+    q = lib.ffd_quantize_keys_tr
+    assert q(ctypes.byref(s), a, a, 0, a, None, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert q(ctypes.byref(s), a, a, 0, a, a + 4, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert q(ctypes.byref(s), a, a, -2, a, a, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert q(ctypes.byref(s), a, a, 64, a, a, a, None) == ffd.FFD_OK  # past the last block
+    s_bad = ffd.make_shape(2, 16, 4, 4096, 32, 16)
+    assert q(ctypes.byref(s_bad), a, a, 0, a, a, a, None) == ffd.FFD_ERR_UNSUPPORTED
+    assert ffd.thumb_bytes(s_bad) == 0 and ffd.residual_bytes(s_bad) == 0
+    # context shards: the pseudo-max is rejected as for the int4 format
+    sink = ffd.DecodeOptions(1, 0)
+    assert lib.ffd_decode_partials_tr(ctypes.byref(s), ctypes.byref(sink), a, a, a, a, a, a, a, 1.0,
+                                      a, ws, None) == ffd.FFD_ERR_UNSUPPORTED
 
 
 def test_product_path_never_touches_the_oracle():
