@@ -195,6 +195,32 @@ def algorithmic_bytes(w, lengths, kept_tokens, dense: bool) -> dict:
             "partials": partials, "total": requant + scan + kv + qo + mask + partials}
 
 
+def algorithmic_bytes_tr(w, lengths, kept_tokens, dense: bool) -> dict:
+    """The same for the thumbnail + residual format: the re-quantisation
+    writes thumbnail (32 B), residual (128 B) rows and scales; the scan reads
+    thumbnails + scales of the valid blocks; the computer reads residuals and
+    V of the kept tokens (their thumbnails and scales were already read by the
+    scan; dense mode reads them here instead of in a scan)."""
+    T, S, G = w.block_size, w.split_blocks, w.group
+    scan = requant = partials = dense_extra = 0
+    for n in lengths:
+        n = int(n)
+        nb = -(-n // T)
+        nsplit = -(-nb // S)
+        if n > 0:
+            requant += w.num_kv_heads * ((n - (nb - 1) * T) * 256 + T * (32 + 128) + 256)
+        if dense:
+            dense_extra += w.num_kv_heads * (n * 32 + nb * 256)
+        else:
+            scan += w.num_kv_heads * (n * 32 + nb * 256)
+        partials += w.num_kv_heads * nsplit * G * 130 * 4 * 2
+    kv = int(kept_tokens) * (128 + 256) + dense_extra
+    qo = 2 * w.batch * w.num_q_heads * 128 * 2
+    mask = w.batch * w.num_kv_heads * math.ceil(w.capacity // T / 32) * 4
+    return {"requant": requant, "scan": scan, "kv": kv, "q_out_mask": qo + mask,
+            "partials": partials, "total": requant + scan + kv + qo + mask + partials}
+
+
 def kept_tokens_from_mask(w, lengths, mask) -> tuple:
     T = w.block_size
     nblk = w.capacity // T
@@ -231,11 +257,12 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic_per_launch(workload: str, dense: bool):
+def ncu_traffic_per_launch(workload: str, dense: bool, fmt: str = "int4"):
     """DRAM bytes per decode launch from the committed ncu summary, if it was
     taken on the current kernel sources (else None)."""
     mode = "dense" if dense else "sparse"
-    path = os.path.join(ROOT, "profiles", f"decode_{workload}_ncu.md")
+    prefix = "decode_tr" if fmt == "tr" else "decode"
+    path = os.path.join(ROOT, "profiles", f"{prefix}_{workload}_ncu.md")
     try:
         text = open(path).read()
     except OSError:
@@ -249,13 +276,14 @@ def ncu_traffic_per_launch(workload: str, dense: bool):
 # ------------------------------------------------------------------ GPU arm --
 
 class Replica:
-    """One GPU's copy of the workload: R rotated layer copies of the cache."""
+    """One GPU's copy of the workload: R rotated layer copies of the cache,
+    with the int4 scan copy ("int4") or thumbnails + residuals ("tr")."""
 
-    def __init__(self, w, inp, device, layers):
+    def __init__(self, w, inp, device, layers, fmt="int4"):
         import torch
         from sparse_long_context_ffd_b200 import ffd
         self.torch, self.ffd = torch, ffd
-        self.w, self.device = w, device
+        self.w, self.device, self.fmt = w, device, fmt
         self.shape = ffd.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.capacity,
                                     w.block_size, w.split_blocks)
 
@@ -267,11 +295,18 @@ class Replica:
         self.lengths = torch.from_numpy(np.ascontiguousarray(inp["lengths"])).to(device)
         self.layers = []
         for i in range(layers):
-            bufs = ffd.DecodeBuffers(self.shape, device=device)
+            if fmt == "tr":
+                bufs = ffd.ThumbResidBuffers(self.shape, device=device)
+            else:
+                bufs = ffd.DecodeBuffers(self.shape, device=device)
             layer = dict(q=q0 if i == 0 else q0.clone(), k=k0 if i == 0 else k0.clone(),
                          v=v0 if i == 0 else v0.clone(), bufs=bufs)
-            ffd.quantize_keys(self.shape, layer["k"], self.lengths, 0, bufs.k_packed,
-                              bufs.k_scales)
+            if fmt == "tr":
+                ffd.quantize_keys_tr(self.shape, layer["k"], self.lengths, 0, bufs.k_thumb,
+                                     bufs.k_resid, bufs.k_scales)
+            else:
+                ffd.quantize_keys(self.shape, layer["k"], self.lengths, 0, bufs.k_packed,
+                                  bufs.k_scales)
             self.layers.append(layer)
         torch.cuda.synchronize(device)
 
@@ -283,14 +318,24 @@ class Replica:
         ffd_decode) when fused is False."""
         L = self.layers[i % len(self.layers)]
         b = L["bufs"]
+        tr = self.fmt == "tr"
         if not fused:
-            self.ffd.quantize_keys(self.shape, L["k"], self.lengths, self.ffd.FFD_LAST_BLOCK,
-                                   b.k_packed, b.k_scales)
+            if tr:
+                self.ffd.quantize_keys_tr(self.shape, L["k"], self.lengths, self.ffd.FFD_LAST_BLOCK,
+                                          b.k_thumb, b.k_resid, b.k_scales)
+            else:
+                self.ffd.quantize_keys(self.shape, L["k"], self.lengths, self.ffd.FFD_LAST_BLOCK,
+                                       b.k_packed, b.k_scales)
         if ev is not None:
             ev[0].record()
-        self.ffd.decode_ex(self.shape, L["q"], L["k"], L["v"], b.k_packed, b.k_scales,
-                           self.lengths, delta, b.out, b.mask, b.workspace,
-                           reference=self.reference, requant_last=fused)
+        if tr:
+            self.ffd.decode_tr(self.shape, L["q"], L["k"], L["v"], b.k_thumb, b.k_resid, b.k_scales,
+                               self.lengths, delta, b.out, b.mask, b.workspace,
+                               reference=self.reference, requant_last=fused)
+        else:
+            self.ffd.decode_ex(self.shape, L["q"], L["k"], L["v"], b.k_packed, b.k_scales,
+                               self.lengths, delta, b.out, b.mask, b.workspace,
+                               reference=self.reference, requant_last=fused)
         if ev is not None:
             ev[1].record()
 
@@ -523,13 +568,14 @@ def run_profile(args):
     w = fw.WORKLOADS[args.workload]
     delta = w.delta if args.delta is None else args.delta
     inp = fw.make_inputs(w)
-    rep = Replica(w, inp, device, 1)
+    rep = Replica(w, inp, device, 1, fmt=args.profile_format)
     rep.reference = REFERENCES[args.reference]
     for i in range(args.profile_steps):
         rep.step(i, delta)
     torch.cuda.synchronize(device)
     rep.check_flags()
-    print(f"profile: {args.profile_steps} eager steps of {w.name} (delta {delta}) done")
+    print(f"profile: {args.profile_steps} eager steps of {w.name} ({args.profile_format}, "
+          f"delta {delta}) done")
     return 0
 
 
@@ -597,6 +643,48 @@ def run_shard_measure(args):
     return 0
 
 
+def measure_thumb_resid(w, inp, device, args, world, l2):
+    """The same decode step on the thumbnail + residual key format (2-bit
+    thumbnails scanned, 8-bit residuals + V read for kept blocks): fused step,
+    dense mode, and its own kept set (the thumbnail scores select differently)."""
+    import torch
+    probe = Replica(w, inp, device, 1, fmt="tr")
+    probe.reference = REFERENCES[args.reference]
+    probe.step(0, w.delta)
+    torch.cuda.synchronize(device)
+    mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
+    kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+    algo = algorithmic_bytes_tr(w, inp["lengths"], kept_tok, dense=False)
+    valid_tok = int(np.sum(inp["lengths"])) * w.num_kv_heads
+    algo_dense = algorithmic_bytes_tr(w, inp["lengths"], valid_tok, dense=True)
+    layers = max(1, min(64, math.ceil(3 * l2 / min(algo["total"], algo_dense["total"]))))
+    del probe
+    rep = Replica(w, inp, device, layers, fmt="tr")
+    rep.reference = REFERENCES[args.reference]
+    steps = min(args.steps, 1000)
+    total, per, _ = time_graph_steps(rep, w.delta, steps, args.warmup, world, device)
+    dense_total, dense_per, _ = time_graph_steps(rep, float("inf"), min(steps, 400),
+                                                 min(args.warmup, 20), world, device)
+    rep.check_flags()
+    peak, _ = load_peaks()
+    dec = float(np.mean(per)) if per else None
+    dden = float(np.mean(dense_per)) if dense_per else None
+    ach = algo["total"] / (dec * 1e-3) / 1e9 if dec else None
+    return {
+        "ms_per_step": dist_max(total / steps, world, device),
+        "decode_us": dec * 1e3 if dec else None,
+        "kept_blocks": kept_blocks, "kept_fraction": kept_blocks / max(1, valid_blocks),
+        "algorithmic_bytes_per_launch": algo, "achieved_gbs": ach,
+        "frac": ach / peak if ach else None,
+        "traffic": ncu_traffic_per_launch(args.workload, dense=False, fmt="tr"),
+        "dense_decode_us": dden * 1e3 if dden else None,
+        "dense_algorithmic_bytes_per_launch": algo_dense["total"],
+        "dense_achieved_gbs": algo_dense["total"] / (dden * 1e-3) / 1e9 if dden else None,
+        "how": "ffd_decode_tr with requant_last (thumbnail + residual re-quantisation of the "
+               "last block + thumbnail scan + residual/V computer + merge), one launch",
+    }
+
+
 def run_gpu(args):
     import torch
     rank, local_rank, world = dist_env()
@@ -659,6 +747,10 @@ def run_gpu(args):
     achieved = algo["total"] / (decode_ms * 1e-3) / 1e9
     traffic = ncu_traffic_per_launch(args.workload, dense=False)
 
+    tr = None
+    if not args.no_tr:
+        tr = measure_thumb_resid(w, inp, device, args, world, l2)
+
     e2e = None
     if not args.no_e2e:
         del rep
@@ -704,6 +796,7 @@ def run_gpu(args):
                            "algorithmic_bytes_per_launch": algo_dense["total"],
                            "achieved_gbs": (algo_dense["total"] / (dense_decode_ms * 1e-3) / 1e9)
                            if dense_decode_ms else None},
+            "thumb_residual": tr,
             "e2e": ({"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                      "d2h_bytes_per_step": e2e["d2h"],
                      "wall_ms_per_step": e2e["wall_ms_per_step"],
@@ -712,6 +805,8 @@ def run_gpu(args):
                             "D2H out+mask, stream sync"} if e2e else None),
             "cpu_baseline": cpu,
             "gpu_launches": args.steps,
+            "gpu_launches_note": "one fused decode launch per timed step (the headline int4 "
+                                 "path); the comparison legs run outside that window",
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -735,12 +830,16 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tr", action="store_true",
+                    help="skip the thumbnail + residual format measurement")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--reference-budget", type=float, default=150.0)
     ap.add_argument("--shards", type=int, default=0,
                     help="time one rank's share of a context-sharded step over this many shards")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps and exit (for ncu)")
+    ap.add_argument("--profile-format", choices=["int4", "tr"], default="int4",
+                    help="key format of the --profile-steps run")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
