@@ -54,6 +54,8 @@ constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kKvTok = kKvBoxRows;                  // tokens per attention stage
 constexpr int kKvHalfBytes = kKvTok * 128;          // one 64-channel half of K or V
 constexpr int kMergeBytes = kAttnWarps * (8 + 8 + 8 * kHeadDim) * 4;
+// block quantiser scratch for the attention warps: per-warp channel maxima + scales
+constexpr int kRequantScratchBytes = (kAttnWarps + 1) * kHeadDim * 4;
 
 // One attention stage (kKvTok tokens of one kept block) per key format.
 template <int F>
@@ -94,8 +96,9 @@ struct SmemLayout {
   static constexpr int kNumBars = 2 * ScanGeom<T, F>::kStages + 2 * NKV;
   static constexpr int kMeta = kBars + 8 * kNumBars;  // int [NKV] token offsets
   static constexpr int kSeq = kMeta + 4 * NKV;        // int [NKV] item indices
-  static constexpr int kCtrl = kSeq + 4 * NKV;        // qcount, sel_done, is_last, abort
-  static constexpr int kKeep = kCtrl + 16;            // u32 [split_words]
+  static constexpr int kCtrl = kSeq + 4 * NKV;        // qcount, sel_done, is_last, abort, requant_done
+  static constexpr int kRequant = kCtrl + 32;         // re-quantisation scratch (attention warps)
+  static constexpr int kKeep = kRequant + kRequantScratchBytes;  // u32 [split_words]
   // queue of kept block indices (u16 [split_blocks]) follows keep bits
 };
 
@@ -379,7 +382,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t *empty_b = full_b + NKV;
   volatile int *meta = reinterpret_cast<volatile int *>(smem + SL::kMeta);
   volatile int *seq = reinterpret_cast<volatile int *>(smem + SL::kSeq);
-  volatile int *ctrl = reinterpret_cast<volatile int *>(smem + SL::kCtrl);  // qcount, done, last, abort
+  // qcount, sel_done, is_last, abort, requant_done
+  volatile int *ctrl = reinterpret_cast<volatile int *>(smem + SL::kCtrl);
   uint32_t *keepbits = reinterpret_cast<uint32_t *>(smem + SL::kKeep);
   volatile uint16_t *queue =
       reinterpret_cast<volatile uint16_t *>(keepbits + ((p.split_words + 3) & ~3));
@@ -431,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     ctrl[1] = 0;
     ctrl[2] = 0;
     ctrl[3] = 0;
+    ctrl[4] = 0;
     fence_mbar_init();
   }
   for (int w = threadIdx.x; w < p.split_words; w += blockDim.x) keepbits[w] = 0u;
@@ -439,29 +444,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     prefetch_tmap(&tmap_v);
   }
   // Fused decode step: the CTA that owns a sequence's last block re-quantises
-  // it (the appended token changed it) before anything reads the int4 copy;
-  // the generic-proxy stores are fenced before the bulk copies read them.
-  if (p.requant_last && split == nsplit - 1) {
-    if (threadIdx.x < kAttnThreads) {
-      const int jl = nb - 1;
-      const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
-      float *red = reinterpret_cast<float *>(scan_ring);  // idle until the scan starts
-      uint16_t *scale_row = p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim;
-      if constexpr (kTR)
-        quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
-                                           p.packed_out + tok0 * kThumbRowBytes,
-                                           p.resid_out + tok0 * kResidRowBytes, scale_row, red,
-                                           red + (kAttnThreads / 32) * kHeadDim,
-                                           static_cast<int>(threadIdx.x), 2);
-      else
-        quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
-                                        p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
-                                        red + (kAttnThreads / 32) * kHeadDim,
-                                        static_cast<int>(threadIdx.x), 2);
-      fence_proxy_async_global();
-    }
-    fence_proxy_async_smem();
-  }
+  // it (the appended token changed it).  The attention warps do it while the
+  // producer and the scan already stream the split's other blocks; only the
+  // copies that read the rewritten block wait for the requant_done flag.
+  const bool owner_requant = p.requant_last && split == nsplit - 1;
   __syncthreads();
 
   // ================================================================ producer
@@ -476,6 +462,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     int q_ptr = 0, sub = 0;         // position in the kept-block list
     int ends_sent = 0;
     uint64_t idle_since = 0;
+    // copies that read the last block's re-quantised data wait for the
+    // attention warps' flag; seeing it, the producer orders their generic
+    // stores before its own async-proxy reads
+    bool requant_seen = !owner_requant;
+    auto requant_ready = [&]() {
+      if (!requant_seen && ctrl[4] != 0) {
+        __threadfence_block();
+        fence_proxy_async_global();
+        requant_seen = true;
+      }
+      return requant_seen;
+    };
     while (true) {
       bool progress = false;
       // scan tiles
@@ -486,8 +484,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         const int st = sc_next % NSA;
         const int use = sc_next / NSA;
-        if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
         const int jb = scan_block_index(sc_next, nref, nb, j0);
+        if (jb == nb - 1 && !requant_ready()) break;
+        if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
         uint8_t *dst = scan_ring + st * SG::kStageBytes;
         mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
         bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * SG::kRowBytes, T * SG::kRowBytes,
@@ -509,6 +508,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           sub = 0;
           continue;
         }
+        // (the int4 computer reads bf16 K/V, which the re-quantisation leaves alone)
+        if (kTR && j0 + j == nb - 1 && !requant_ready()) break;
         const int st = it_next % NKV;
         const int use = it_next / NKV;
         if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
@@ -662,6 +663,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         qb[ks][1] = gid < G ? qh[8 * ks + 4 + t4] : 0u;
       }
     }
+  }
+  if (owner_requant) {
+    // the last block's re-quantisation (see the prologue); the stores are
+    // fenced for the async proxy before the flag releases the producer
+    const int jl = nb - 1;
+    const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
+    float *red = reinterpret_cast<float *>(smem + SL::kRequant);
+    uint16_t *scale_row = p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim;
+    if constexpr (kTR)
+      quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                         p.packed_out + tok0 * kThumbRowBytes,
+                                         p.resid_out + tok0 * kResidRowBytes, scale_row, red,
+                                         red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2);
+    else
+      quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                      p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
+                                      red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2);
+    fence_proxy_async_global();
+    __threadfence_block();
+    named_barrier(2, kAttnThreads);
+    if (threadIdx.x == 0) ctrl[4] = 1;
   }
   if (local_in_smem) {
     // Quantise the local block from K into scan stage 1 (the producer skips
