@@ -942,6 +942,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       bits = lo >= nbs ? 0u : (nbs - lo >= 32 ? kFull : ((1u << (nbs - lo)) - 1u));
     }
     p.split_bits[unit * p.split_words + threadIdx.x] = bits;
+    // splits of a multiple of 32 blocks own whole mask words: write them here
+    // rather than gather them in the final merge
+    if (!p.partials_only && (p.split_blocks & 31) == 0 && (j0 >> 5) + static_cast<int>(threadIdx.x) < p.mask_words)
+      p.mask[row * p.mask_words + (j0 >> 5) + threadIdx.x] = bits;
+  }
+  if (!p.partials_only && (p.split_blocks & 31) == 0 && split == nsplit - 1) {
+    // the last split also clears the words past its range
+    for (int w = ((j0 + p.split_blocks) >> 5) + static_cast<int>(threadIdx.x); w < p.mask_words; w += kAttnThreads)
+      p.mask[row * p.mask_words + w] = 0u;
   }
   if (p.partials_only) return;  // context shard: the merge runs after the exchange
   __threadfence();
@@ -952,108 +961,71 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (!ctrl[2]) return;
   __threadfence();
 
-  // last CTA of (b, g): log-sum-exp merge over the splits.  Every load here
-  // is independent of the others, so the merge costs about three L2 round
-  // trips rather than one per split:
-  //   1. per head (one warp per head, lanes striding over the splits): the
-  //      split maxima and sums are combined pairwise, (m1, l1) + (m2, l2) =
-  //      (M, l1 2^(m1 - M) + l2 2^(m2 - M)), into M* and L*; the split maxima
-  //      of the first chunk stay in shared memory;
-  //   2. per chunk of splits: weights 2^(m_s - M*) / L* in shared memory,
-  //      then each thread accumulates four output channels with float4 loads
-  //      issued sixteen at a time.
+  // last CTA of (b, g): log-sum-exp merge over the splits.  Warp w merges
+  // heads w, w + 4 (lane: output channels 4*lane .. 4*lane + 3).  Per chunk of
+  // 16 splits every load (m, l and the lane's float4 of acc) is independent of
+  // the others, so the merge costs about one L2 round trip per chunk; the
+  // chunk is folded into a running (M, L, O) with the pairwise rule
+  // (m1, l1, o1) + (m2, l2, o2) = (M, l1 2^(m1 - M) + l2 2^(m2 - M),
+  // o1 2^(m1 - M) + o2 2^(m2 - M)), M = max(m1, m2).  A split that kept no
+  // token has m = -inf and is skipped.
   const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
-  float *stats = reinterpret_cast<float *>(scan_ring);  // [G][2]: M*, L*
-  float *wts = stats + 16;                              // [chunk][G]
-  constexpr int kWtsFloats = SG::kRingBytes / 4 - 16;
-  const int chunk = kWtsFloats / G;
+  constexpr int kChunk = 16;
   for (int h = warp; h < G; h += kAttnWarps) {
-    float m = -INFINITY, l = 0.0f;
-    for (int s = lane; s < nsplit; s += 32) {
-      const float *ps = row_parts + (s * G + h) * kPartialStride;
-      const float ms = __ldcg(ps + 128), ls = __ldcg(ps + 129);
-      if (s < chunk) wts[s * G + h] = ms;
-      const float mn = fmaxf(m, ms);  // -inf only while no split so far kept a token
-      if (mn != -INFINITY) {
-        l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (ms == -INFINITY ? 0.0f : ls * exp2f(ms - mn));
-        m = mn;
-      }
-    }
+    float M = -INFINITY, L = 0.0f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nsplit; s0 += kChunk) {
+      float ms[kChunk], ls[kChunk];
+      float4 v[kChunk];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float mo = __shfl_xor_sync(kFull, m, off), lo = __shfl_xor_sync(kFull, l, off);
-      const float mn = fmaxf(m, mo);
-      if (mn != -INFINITY) {
-        l = (m == -INFINITY ? 0.0f : l * exp2f(m - mn)) + (mo == -INFINITY ? 0.0f : lo * exp2f(mo - mn));
-        m = mn;
-      }
-    }
-    if (lane == 0) {
-      stats[2 * h] = m;
-      stats[2 * h + 1] = l;
-    }
-  }
-  named_barrier(1, kAttnThreads);
-  const int f = threadIdx.x;  // float4 output index: head f / 32, channels 4 (f % 32) ..
-  float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;  // second set for G == 8
-  for (int s0 = 0; s0 < nsplit; s0 += chunk) {
-    const int cnt = min(chunk, nsplit - s0);
-    for (int i = threadIdx.x; i < cnt * G; i += kAttnThreads) {
-      const int h = i % G, s = s0 + i / G;
-      const float ms = s0 == 0 ? wts[i] : __ldcg(row_parts + (s * G + h) * kPartialStride + 128);
-      wts[i] = ms == -INFINITY ? 0.0f : exp2f(ms - stats[2 * h]) / stats[2 * h + 1];
-    }
-    named_barrier(1, kAttnThreads);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int fi = f + half * kAttnThreads;
-      if (fi < G * 32) {
-        const int h = fi >> 5, c4 = fi & 31;
-        float4 acc = half ? o1 : o0;
-        int s = 0;
-        for (; s + 16 <= cnt; s += 16) {
-          float4 v[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            v[u] = __ldcg(reinterpret_cast<const float4 *>(row_parts + ((s0 + s + u) * G + h) * kPartialStride) + c4);
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float wgt = wts[(s + u) * G + h];
-            acc.x += wgt * v[u].x;
-            acc.y += wgt * v[u].y;
-            acc.z += wgt * v[u].z;
-            acc.w += wgt * v[u].w;
-          }
+      for (int u = 0; u < kChunk; ++u) {
+        if (s0 + u < nsplit) {
+          const float *ps = row_parts + ((s0 + u) * G + h) * kPartialStride;
+          ms[u] = __ldcg(ps + 128);
+          ls[u] = __ldcg(ps + 129);
+          v[u] = __ldcg(reinterpret_cast<const float4 *>(ps) + lane);
+        } else {
+          ms[u] = -INFINITY;
+          ls[u] = 0.0f;
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (; s < cnt; ++s) {
-          const float4 v = __ldcg(reinterpret_cast<const float4 *>(row_parts + ((s0 + s) * G + h) * kPartialStride) + c4);
-          const float wgt = wts[s * G + h];
-          acc.x += wgt * v.x;
-          acc.y += wgt * v.y;
-          acc.z += wgt * v.z;
-          acc.w += wgt * v.w;
-        }
-        if (half) o1 = acc; else o0 = acc;
       }
-    }
-    named_barrier(1, kAttnThreads);
-  }
+      float mc = M;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int fi = f + half * kAttnThreads;
-    if (fi < G * 32) {
-      const float4 acc = half ? o1 : o0;
-      const uint32_t lo = pack_bf16x2(acc.x, acc.y), hi = pack_bf16x2(acc.z, acc.w);
-      *reinterpret_cast<uint2 *>(out_rows + (fi >> 5) * kHeadDim + 4 * (fi & 31)) = make_uint2(lo, hi);
+      for (int u = 0; u < kChunk; ++u) mc = fmaxf(mc, ms[u]);
+      if (mc == -INFINITY) continue;
+      const float f = M == -INFINITY ? 0.0f : exp2f(M - mc);
+      L *= f;
+      O.x *= f;
+      O.y *= f;
+      O.z *= f;
+      O.w *= f;
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u) {
+        if (ms[u] != -INFINITY) {
+          const float wgt = exp2f(ms[u] - mc);
+          L += ls[u] * wgt;
+          O.x += wgt * v[u].x;
+          O.y += wgt * v[u].y;
+          O.z += wgt * v[u].z;
+          O.w += wgt * v[u].w;
+        }
+      }
+      M = mc;
     }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    const uint32_t lo = pack_bf16x2(O.x * inv, O.y * inv), hi = pack_bf16x2(O.z * inv, O.w * inv);
+    *reinterpret_cast<uint2 *>(out_rows + h * kHeadDim + 4 * lane) = make_uint2(lo, hi);
   }
-  // mask row: each word gathers 32 consecutive blocks' bits from the split
-  // bit rows
-  const uint32_t *row_bits = p.split_bits + row * p.nsplit_max * p.split_words;
-  const int split_words = p.split_words;
-  for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads)
-    p.mask[row * p.mask_words + w] = gather_mask_word(
-        w, nb, p.split_blocks, [&](int s, int wd) { return __ldcg(row_bits + s * split_words + wd); });
+  // mask row (splits not a multiple of 32 blocks): each word gathers 32
+  // consecutive blocks' bits from the split bit rows
+  if ((p.split_blocks & 31) != 0) {
+    const uint32_t *row_bits = p.split_bits + row * p.nsplit_max * p.split_words;
+    const int split_words = p.split_words;
+    for (int w = threadIdx.x; w < p.mask_words; w += kAttnThreads)
+      p.mask[row * p.mask_words + w] = gather_mask_word(
+          w, nb, p.split_blocks, [&](int s, int wd) { return __ldcg(row_bits + s * split_words + wd); });
+  }
   if (threadIdx.x == 0) p.counters[row] = 0u;
 }
 

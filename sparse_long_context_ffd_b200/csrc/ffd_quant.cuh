@@ -110,9 +110,11 @@ __device__ __forceinline__ void quantize_block(const uint16_t *k_rows, int valid
 //
 // NT threads quantise one block of T rows.  Thread (rg = tid / 8, cg = tid % 8)
 // owns channels 16cg .. 16cg+15 (thumbnail word cg, residual bytes 16cg ..) of
-// rows rg, rg + NT/8, ...; the rows are read twice (amax pass, then codes) so
-// that no row lives in registers across the barrier.  resid_rows may be null
-// (a scan-only copy).  red holds NT/32 x 128 floats, scale_s 128 floats.
+// rows rg, rg + NT/8, ...  Rows are loaded four at a time with all loads in
+// flight together; up to four rows per thread stay in registers between the
+// amax pass and the code pass, more are re-read (from L1/L2) four at a time.
+// resid_rows may be null (a scan-only copy).  red holds NT/32 x 128 floats,
+// scale_s 128 floats.
 template <int T, int NT>
 __device__ __forceinline__ void quantize_block_tr(const uint16_t *k_rows, int valid, uint8_t *thumb_rows,
                                                   uint8_t *resid_rows, uint16_t *scale_row, float *red,
@@ -120,20 +122,34 @@ __device__ __forceinline__ void quantize_block_tr(const uint16_t *k_rows, int va
   static_assert(NT % 32 == 0 && NT >= 32 && T % (NT / 8) == 0, "thread layout");
   constexpr int RG = NT / 8;  // row groups
   constexpr int R = T / RG;   // rows per thread
+  constexpr int RC = R < 4 ? R : 4;  // rows per load round
   const int cg = tid & 7;
   const int rg = tid >> 3;
+  uint4 x[RC][2];
+  auto load_rows = [&](int r0) {
+#pragma unroll
+    for (int i = 0; i < RC; ++i) {
+      const int t = rg + RG * (r0 + i);
+      if (t < valid) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 16 * cg);
+        x[i][0] = src[0];
+        x[i][1] = src[1];
+      } else {
+        x[i][0] = x[i][1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  };
   float amax[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) amax[c] = 0.0f;
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const int t = rg + RG * r;
-    if (t < valid) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 16 * cg);
+  for (int r0 = 0; r0 < R; r0 += RC) {
+    load_rows(r0);
+#pragma unroll
+    for (int i = 0; i < RC; ++i) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint4 x = src[h];
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        const uint32_t w[4] = {x[i][h].x, x[i][h].y, x[i][h].z, x[i][h].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           amax[8 * h + 2 * e] = fmaxf(amax[8 * h + 2 * e], fabsf(q_bf16_lo(w[e])));
@@ -166,15 +182,16 @@ __device__ __forceinline__ void quantize_block_tr(const uint16_t *k_rows, int va
   float sf[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) sf[c] = scale_s[16 * cg + c];
-#pragma unroll 1
+#pragma unroll
   for (int r = 0; r < R; ++r) {
+    const int i = r % RC;
+    if (R > RC && i == 0) load_rows(r);
     const int t = rg + RG * r;
     uint32_t word = 0u;
     uint32_t rb[4] = {0u, 0u, 0u, 0u};
     if (t < valid) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 16 * cg);
-      const uint4 x0 = src[0], x1 = src[1];
-      const uint32_t w[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const uint32_t w[8] = {x[i][0].x, x[i][0].y, x[i][0].z, x[i][0].w,
+                             x[i][1].x, x[i][1].y, x[i][1].z, x[i][1].w};
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const float v = (c & 1) ? q_bf16_hi(w[c >> 1]) : q_bf16_lo(w[c >> 1]);

@@ -31,6 +31,9 @@ SMALL = [
     (7, 2, 4, 1, 4096, 64, 33, 1, 4096),
     (8, 1, 4, 1, 2048, 64, 1, 2048, 2048),
     (9, 2, 2, 1, 8192, 128, 40, 3000, 8192),
+    # splits of a multiple of 32 blocks whose last split overhangs the capacity
+    (10, 2, 4, 2, 4480, 64, 64, 1, 4480),
+    (11, 3, 2, 1, 12800, 128, 32, 1, 12800),
 ]
 
 

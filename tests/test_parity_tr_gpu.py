@@ -27,6 +27,7 @@ SMALL = [
     (5, 3, 8, 2, 4096, 128, 7, 100, 4096),
     (6, 1, 4, 2, 8192, 64, 64, 5000, 8192),
     (7, 2, 4, 1, 4096, 64, 33, 1, 4096),
+    (10, 2, 4, 2, 4480, 64, 64, 1, 4480),
 ]
 
 THUMB_POISON = 0x5A
