@@ -422,9 +422,10 @@ def time_gated_decodes(rep, delta, n, device):
 
 
 def e2e_steps(w, inp, device, delta, steps):
-    """End-to-end decode steps through the public API with host buffers:
-    H2D of the step's query and new key/value rows from pinned memory, the
-    append into the cache, quantise + decode, D2H of output and mask."""
+    """End-to-end decode steps through the public API with host buffers: one
+    pinned H2D copy of the step's query and new key/value rows, one fused
+    launch (append into the cache + last-block re-quantisation + decode,
+    ffd_decode_append), D2H of output and mask."""
     import torch
     from sparse_long_context_ffd_b200 import ffd
     shape = ffd.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.capacity, w.block_size,
@@ -440,27 +441,25 @@ def e2e_steps(w, inp, device, delta, steps):
     bufs = ffd.DecodeBuffers(shape, device=device)
     ffd.quantize_keys(shape, k, lengths, 0, bufs.k_packed, bufs.k_scales)
     B, Hq, Hkv, D = w.batch, w.num_q_heads, w.num_kv_heads, 128
-    # pinned host inputs: per step the query and the newest token's K/V rows
-    host_in = torch.empty((B, Hq + 2 * Hkv, D), dtype=torch.bfloat16).pin_memory()
-    host_in[:, :Hq] = bf16(inp["q"])
-    pos = torch.from_numpy((lengths_h - 1).astype(np.int64))
-    for b in range(B):
-        host_in[b, Hq:Hq + Hkv] = bf16(inp["k"][b, :, int(lengths_h[b]) - 1])
-        host_in[b, Hq + Hkv:] = bf16(inp["v"][b, :, int(lengths_h[b]) - 1])
+    # pinned host inputs, one flat buffer: q [B,Hq,D] | k_new [B,Hkv,D] | v_new [B,Hkv,D]
+    nq, nk = B * Hq * D, B * Hkv * D
+    host_in = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
+    host_in[:nq] = bf16(inp["q"]).reshape(-1)
+    last = [int(lengths_h[b]) - 1 for b in range(B)]
+    host_in[nq:nq + nk] = torch.stack([bf16(inp["k"][b, :, last[b]]) for b in range(B)]).reshape(-1)
+    host_in[nq + nk:] = torch.stack([bf16(inp["v"][b, :, last[b]]) for b in range(B)]).reshape(-1)
     dev_in = torch.empty_like(host_in, device=device)
+    q_d = dev_in[:nq].view(B, Hq, D)
+    k_new = dev_in[nq:nq + nk].view(B, Hkv, D)
+    v_new = dev_in[nq + nk:].view(B, Hkv, D)
     host_out = torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory()
     host_mask = torch.empty(bufs.mask.shape, dtype=torch.int32).pin_memory()
-    bidx = torch.arange(B, device=device)
-    pos_d = pos.to(device)
     stream = torch.cuda.current_stream(device)
 
     def one():
         dev_in.copy_(host_in, non_blocking=True)
-        q = dev_in[:, :Hq]
-        k[bidx, :, pos_d] = dev_in[:, Hq:Hq + Hkv]
-        v[bidx, :, pos_d] = dev_in[:, Hq + Hkv:]
-        ffd.decode_step(shape, q.contiguous(), k, v, bufs.k_packed, bufs.k_scales, lengths,
-                        delta, bufs.out, bufs.mask, bufs.workspace)
+        ffd.decode_append(shape, q_d, k_new, v_new, k, v, bufs.k_packed, bufs.k_scales, lengths,
+                          delta, bufs.out, bufs.mask, bufs.workspace)
         host_out.copy_(bufs.out, non_blocking=True)
         host_mask.copy_(bufs.mask, non_blocking=True)
         stream.synchronize()
@@ -800,9 +799,9 @@ def run_gpu(args):
             "e2e": ({"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                      "d2h_bytes_per_step": e2e["d2h"],
                      "wall_ms_per_step": e2e["wall_ms_per_step"],
-                     "how": "public Python API per step: pinned H2D of q + new K/V rows, "
-                            "cache append, decode_step (last-block re-quantisation + decode), "
-                            "D2H out+mask, stream sync"} if e2e else None),
+                     "how": "public Python API per step: one pinned H2D of q + new K/V rows, "
+                            "decode_append (cache append + last-block re-quantisation + decode "
+                            "in one launch), D2H out+mask, stream sync"} if e2e else None),
             "cpu_baseline": cpu,
             "gpu_launches": args.steps,
             "gpu_launches_note": "one fused decode launch per timed step (the headline int4 "

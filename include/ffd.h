@@ -238,6 +238,33 @@ ffd_status ffd_decode_tr(const ffd_shape *shape, const ffd_decode_options *optio
                          void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
                          void *cuda_stream);
 
+/* ---- The decode step with the KV append fused in ----
+ * One launch per decode step for callers that hold the new token's K and V
+ * rows (k_new, v_new: bf16 [B][Hkv][D]) rather than an already appended
+ * cache: the CTA that owns each sequence's last block writes the two rows
+ * into k and v at position lengths[b] - 1 (lengths[b] counts the new token),
+ * re-quantises that block and runs the decode; every CTA that reads the new
+ * token takes it from k_new, so nothing waits on another CTA.  Equivalent to
+ * storing the rows, then ffd_decode_step (or ffd_decode_ex with requant_last
+ * and `reference`; ffd_decode_tr for the _tr form); the results are
+ * bit-identical.  The step of the pages' system part (gist.science explainer,
+ * Methodology 3: the decoding step captured whole in a CUDA graph) keeps one
+ * kernel per layer this way.  reference: FFD_REFERENCE_*.  A sequence of
+ * length 0 appends nothing.  Other arguments and errors as ffd_decode_ex and
+ * ffd_decode_tr. */
+ffd_status ffd_decode_append(const ffd_shape *shape, int32_t reference, const void *q_bf16,
+                             const void *k_new_bf16, const void *v_new_bf16, void *k_bf16,
+                             void *v_bf16, void *k_packed, void *k_scales,
+                             const int32_t *d_lengths, float delta, void *out_bf16,
+                             uint32_t *mask, void *workspace, size_t workspace_bytes,
+                             void *cuda_stream);
+ffd_status ffd_decode_append_tr(const ffd_shape *shape, int32_t reference, const void *q_bf16,
+                                const void *k_new_bf16, const void *v_new_bf16, void *k_bf16,
+                                void *v_bf16, void *k_thumb, void *k_resid, void *k_scales,
+                                const int32_t *d_lengths, float delta, void *out_bf16,
+                                uint32_t *mask, void *workspace, size_t workspace_bytes,
+                                void *cuda_stream);
+
 /* Context (sequence) sharding across GPUs.  Each rank holds a contiguous
  * shard of every sequence's cache: rank r holds global tokens
  * [r * cap_local, (r + 1) * cap_local) in a cache of capacity cap_local, with

@@ -245,10 +245,13 @@ struct KeyBuffers {
 };
 
 // Shared body of every decode entry point.
+// k_new / v_new (bf16 [B][Hkv][D], both or neither): the fused append writes
+// them into the caches at position length - 1 (requant must be set).
 ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffers &kb, const void *v_bf16,
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
-                         int32_t reference, bool partials_only = false) {
+                         int32_t reference, bool partials_only = false, const void *k_new = nullptr,
+                         const void *v_new = nullptr) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL)
@@ -278,6 +281,10 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   if (need_k && kb.k == nullptr) return FFD_ERR_INVALID_ARG;
   if (need_packed && (kb.packed == nullptr || kb.scales == nullptr)) return FFD_ERR_INVALID_ARG;
   if (tr && kb.resid == nullptr) return FFD_ERR_INVALID_ARG;
+  const bool append = k_new != nullptr || v_new != nullptr;
+  if (append && (k_new == nullptr || v_new == nullptr || kb.k == nullptr || !requant ||
+                 !aligned16(k_new) || !aligned16(v_new)))
+    return FFD_ERR_INVALID_ARG;
   if (!aligned16(q_bf16) || !aligned16(kb.k) || !aligned16(v_bf16) || !aligned16(out_bf16) ||
       !aligned16(mask) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(d_lengths) & 3u) != 0)
     return FFD_ERR_INVALID_ARG;  // (null pointers pass: aligned16(nullptr) holds)
@@ -316,6 +323,10 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(kb.packed)) : nullptr;
   p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(kb.scales)) : nullptr;
   p.resid_out = requant && tr ? static_cast<uint8_t *>(const_cast<void *>(kb.resid)) : nullptr;
+  p.k_new = static_cast<const uint16_t *>(k_new);
+  p.v_new = static_cast<const uint16_t *>(v_new);
+  p.k_out = append ? static_cast<uint16_t *>(const_cast<void *>(kb.k)) : nullptr;
+  p.v_out = append ? static_cast<uint16_t *>(const_cast<void *>(v_bf16)) : nullptr;
 
   const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
                   static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
@@ -435,6 +446,26 @@ ffd_status ffd_decode_ex(const ffd_shape *s, const ffd_decode_options *opt, cons
   return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
                        opt->reference);
+}
+
+ffd_status ffd_decode_append(const ffd_shape *s, int32_t reference, const void *q_bf16,
+                             const void *k_new_bf16, const void *v_new_bf16, void *k_bf16, void *v_bf16,
+                             void *k_packed, void *k_scales, const int32_t *d_lengths, float delta,
+                             void *out_bf16, uint32_t *mask, void *workspace, size_t workspace_bytes,
+                             void *cuda_stream) {
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
+                       mask, workspace, workspace_bytes, cuda_stream, true, reference, false, k_new_bf16,
+                       v_new_bf16);
+}
+
+ffd_status ffd_decode_append_tr(const ffd_shape *s, int32_t reference, const void *q_bf16,
+                                const void *k_new_bf16, const void *v_new_bf16, void *k_bf16, void *v_bf16,
+                                void *k_thumb, void *k_resid, void *k_scales, const int32_t *d_lengths,
+                                float delta, void *out_bf16, uint32_t *mask, void *workspace,
+                                size_t workspace_bytes, void *cuda_stream) {
+  return decode_common(s, q_bf16, tr_keys(k_bf16, k_thumb, k_resid, k_scales), v_bf16, d_lengths, delta,
+                       out_bf16, mask, workspace, workspace_bytes, cuda_stream, true, reference, false,
+                       k_new_bf16, v_new_bf16);
 }
 
 ffd_status ffd_decode_tr(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,

@@ -508,8 +508,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           sub = 0;
           continue;
         }
-        // (the int4 computer reads bf16 K/V, which the re-quantisation leaves alone)
-        if (kTR && j0 + j == nb - 1 && !requant_ready()) break;
+        // (the int4 computer reads bf16 K/V, which only the fused append changes)
+        if ((kTR || p.k_new != nullptr) && j0 + j == nb - 1 && !requant_ready()) break;
         const int st = it_next % NKV;
         const int use = it_next / NKV;
         if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
@@ -664,22 +664,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
+  // fused append: the new token's K row (read by the quantisers from k_new,
+  // since this CTA's own cache store is not yet visible to them)
+  const uint16_t *new_k_row = p.k_new != nullptr ? p.k_new + row * kHeadDim : nullptr;
   if (owner_requant) {
-    // the last block's re-quantisation (see the prologue); the stores are
-    // fenced for the async proxy before the flag releases the producer
+    // the last block's re-quantisation (see the prologue), after the append's
+    // cache stores; all stores are fenced for the async proxy before the flag
+    // releases the producer
     const int jl = nb - 1;
     const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
+    if (new_k_row != nullptr && threadIdx.x < 32) {
+      const size_t at = (row * static_cast<size_t>(p.capacity) + static_cast<size_t>(len - 1)) * kHeadDim;
+      const int c = threadIdx.x & 15;
+      if (threadIdx.x < 16)
+        reinterpret_cast<uint4 *>(p.k_out + at)[c] = reinterpret_cast<const uint4 *>(new_k_row)[c];
+      else
+        reinterpret_cast<uint4 *>(p.v_out + at)[c] = reinterpret_cast<const uint4 *>(p.v_new + row * kHeadDim)[c];
+    }
     float *red = reinterpret_cast<float *>(smem + SL::kRequant);
     uint16_t *scale_row = p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim;
     if constexpr (kTR)
       quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
                                          p.packed_out + tok0 * kThumbRowBytes,
                                          p.resid_out + tok0 * kResidRowBytes, scale_row, red,
-                                         red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2);
+                                         red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
+                                         new_k_row);
     else
       quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
                                       p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
-                                      red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2);
+                                      red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
+                                      new_k_row);
     fence_proxy_async_global();
     __threadfence_block();
     named_barrier(2, kAttnThreads);
@@ -697,10 +711,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if constexpr (kTR)
       quantize_block_tr<T, kAttnThreads>(k_rows, min(T, len - jl * T), tile, nullptr, scale_row, red,
                                          red + (kAttnThreads / 32) * kHeadDim,
-                                         static_cast<int>(threadIdx.x), 2);
+                                         static_cast<int>(threadIdx.x), 2, new_k_row);
     else
       quantize_block<T, kAttnThreads>(k_rows, min(T, len - jl * T), tile, scale_row, red,
-                                      red + (kAttnThreads / 32) * kHeadDim, static_cast<int>(threadIdx.x), 2);
+                                      red + (kAttnThreads / 32) * kHeadDim, static_cast<int>(threadIdx.x), 2,
+                                      new_k_row);
     fence_proxy_async_smem();  // both regions are later written by async copies
     named_barrier(2, kAttnThreads);
     if (threadIdx.x == 0) mbar_arrive(&full_a[1]);

@@ -53,6 +53,12 @@ struct DecodeParams {
   uint8_t *packed_out;       // = packed, written for the last block
   uint16_t *scales_out;      // = scales, written for the last block
   uint8_t *resid_out;        // thumbnail format: residuals [B][Hkv][cap][128], last block
+  // fused append: the new token's K and V rows (bf16 [B][Hkv][D]) are written
+  // into the caches at position length - 1 by the CTA owning the last block
+  const uint16_t *k_new;     // null: no append
+  const uint16_t *v_new;
+  uint16_t *k_out;           // = k (the bf16 K cache), written at the new token only
+  uint16_t *v_out;           // = the bf16 V cache, written at the new token only
   // context sharding: write the split partials and bits only (no final merge;
   // out and mask unused)
   int32_t partials_only;

@@ -28,11 +28,12 @@ __device__ __forceinline__ float q_bf16_hi(uint32_t w) { return __uint_as_float(
 // 8cg .. 8cg+7 of rows rg, rg + NT/16, ...: one 16-byte load and one 4-byte
 // store of 8 nibbles per row.  red holds NT/32 x 128 floats and scale_s 128
 // floats of shared memory; `bar_id` names a barrier used by exactly these NT
-// threads.
+// threads.  When last_row is not null it replaces the block's last valid row
+// (the token being appended, not yet visible in k_rows to this CTA).
 template <int T, int NT>
 __device__ __forceinline__ void quantize_block(const uint16_t *k_rows, int valid, uint8_t *packed_rows,
                                                uint16_t *scale_row, float *red, float *scale_s, int tid,
-                                               uint32_t bar_id) {
+                                               uint32_t bar_id, const uint16_t *last_row = nullptr) {
   static_assert(NT % 32 == 0 && NT >= 32 && T % (NT / 16) == 0, "thread layout");
   constexpr int RG = NT / 16;  // row groups
   constexpr int R = T / RG;    // rows per thread
@@ -46,7 +47,9 @@ __device__ __forceinline__ void quantize_block(const uint16_t *k_rows, int valid
   for (int r = 0; r < R; ++r) {
     const int t = rg + RG * r;
     if (t < valid) {
-      x[r] = *reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 8 * cg);
+      const uint16_t *src = (last_row != nullptr && t == valid - 1) ? last_row
+                                                                     : k_rows + static_cast<size_t>(t) * kHeadDim;
+      x[r] = *reinterpret_cast<const uint4 *>(src + 8 * cg);
       const uint32_t w[4] = {x[r].x, x[r].y, x[r].z, x[r].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -114,11 +117,12 @@ __device__ __forceinline__ void quantize_block(const uint16_t *k_rows, int valid
 // flight together; up to four rows per thread stay in registers between the
 // amax pass and the code pass, more are re-read (from L1/L2) four at a time.
 // resid_rows may be null (a scan-only copy).  red holds NT/32 x 128 floats,
-// scale_s 128 floats.
+// scale_s 128 floats.  last_row as for quantize_block.
 template <int T, int NT>
 __device__ __forceinline__ void quantize_block_tr(const uint16_t *k_rows, int valid, uint8_t *thumb_rows,
                                                   uint8_t *resid_rows, uint16_t *scale_row, float *red,
-                                                  float *scale_s, int tid, uint32_t bar_id) {
+                                                  float *scale_s, int tid, uint32_t bar_id,
+                                                  const uint16_t *last_row = nullptr) {
   static_assert(NT % 32 == 0 && NT >= 32 && T % (NT / 8) == 0, "thread layout");
   constexpr int RG = NT / 8;  // row groups
   constexpr int R = T / RG;   // rows per thread
@@ -131,7 +135,9 @@ __device__ __forceinline__ void quantize_block_tr(const uint16_t *k_rows, int va
     for (int i = 0; i < RC; ++i) {
       const int t = rg + RG * (r0 + i);
       if (t < valid) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(k_rows + static_cast<size_t>(t) * kHeadDim + 16 * cg);
+        const uint16_t *row = (last_row != nullptr && t == valid - 1) ? last_row
+                                                                       : k_rows + static_cast<size_t>(t) * kHeadDim;
+        const uint4 *src = reinterpret_cast<const uint4 *>(row + 16 * cg);
         x[i][0] = src[0];
         x[i][1] = src[1];
       } else {

@@ -35,7 +35,7 @@ EXPORTED = (
     "ffd_status_string", "ffd_abi_version", "ffd_decode_no_alloc", "ffd_decode_step",
     "ffd_decode_ex", "ffd_decode_partials", "ffd_partials_region", "ffd_merge_partials",
     "ffd_thumb_bytes", "ffd_residual_bytes", "ffd_quantize_keys_tr", "ffd_decode_tr",
-    "ffd_decode_partials_tr",
+    "ffd_decode_partials_tr", "ffd_decode_append", "ffd_decode_append_tr",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -104,6 +104,13 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_decode_partials_tr.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p,
                                                    p, p, p, ctypes.c_float, p, sz, p]
             lib.ffd_decode_partials_tr.restype = st
+            i32 = ctypes.c_int32
+            lib.ffd_decode_append.argtypes = [sp, i32, p, p, p, p, p, p, p, p, ctypes.c_float, p,
+                                              p, p, sz, p]
+            lib.ffd_decode_append.restype = st
+            lib.ffd_decode_append_tr.argtypes = [sp, i32, p, p, p, p, p, p, p, p, p,
+                                                 ctypes.c_float, p, p, p, sz, p]
+            lib.ffd_decode_append_tr.restype = st
             lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode.restype = st
             lib.ffd_decode_ex.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p,
@@ -221,6 +228,32 @@ def decode_tr(shape: Shape, q, k, v, k_thumb, k_resid, k_scales, lengths, delta:
                                          _ptr(workspace),
                                          workspace.numel() * workspace.element_size(),
                                          _stream(stream)), "ffd_decode_tr")
+
+
+def decode_append(shape: Shape, q, k_new, v_new, k, v, k_packed, k_scales, lengths,
+                  delta: float, out, mask, workspace,
+                  reference: int = FFD_REFERENCE_RUNNING_MAX, stream=None) -> None:
+    """One launch per step: write the new token's K/V rows (k_new, v_new
+    [B,Hkv,D]) at position lengths-1, re-quantise the last block, decode."""
+    _check(load_library().ffd_decode_append(ctypes.byref(shape), int(reference), _ptr(q),
+                                             _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
+                                             _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
+                                             float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(),
+                                             _stream(stream)), "ffd_decode_append")
+
+
+def decode_append_tr(shape: Shape, q, k_new, v_new, k, v, k_thumb, k_resid, k_scales, lengths,
+                     delta: float, out, mask, workspace,
+                     reference: int = FFD_REFERENCE_RUNNING_MAX, stream=None) -> None:
+    """decode_append on the thumbnail + residual key format."""
+    _check(load_library().ffd_decode_append_tr(ctypes.byref(shape), int(reference), _ptr(q),
+                                                _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
+                                                _ptr(k_thumb), _ptr(k_resid), _ptr(k_scales),
+                                                _ptr(lengths), float(delta), _ptr(out), _ptr(mask),
+                                                _ptr(workspace),
+                                                workspace.numel() * workspace.element_size(),
+                                                _stream(stream)), "ffd_decode_append_tr")
 
 
 def decode_partials_tr(local_shape: Shape, q, k, v, k_thumb, k_resid, k_scales, local_lengths,

@@ -166,6 +166,30 @@ def test_thumb_resid_arguments_rejected_on_host():
                                       a, ws, None) == ffd.FFD_ERR_UNSUPPORTED
 
 
+def test_append_arguments_rejected_on_host():
+    lib = ffd.load_library()
+    s = ffd.make_shape(2, 16, 4, 4096, 64, 16)
+    ws = ffd.decode_workspace_bytes(s)
+    a = 1 << 20
+
+    def app(ref=0, q=a, kn=a, vn=a, k=a, v=a, p=a, sc=a, ln=a, delta=1.0):
+        return lib.ffd_decode_append(ctypes.byref(s), ref, q, kn, vn, k, v, p, sc, ln, delta, a, a,
+                                     a, ws, None)
+
+    def app_tr(kn=a, vn=a, k=a, re=a):
+        return lib.ffd_decode_append_tr(ctypes.byref(s), 0, a, kn, vn, k, a, a, re, a, a, 1.0, a, a,
+                                        a, ws, None)
+
+    for name in ("kn", "vn", "k", "v", "p", "sc"):
+        assert app(**{name: None}) == ffd.FFD_ERR_INVALID_ARG, name
+    assert app(kn=a + 4) == ffd.FFD_ERR_INVALID_ARG and app(vn=a + 2) == ffd.FFD_ERR_INVALID_ARG
+    assert app(ref=2) == ffd.FFD_ERR_INVALID_ARG
+    assert app(delta=float("nan")) == ffd.FFD_ERR_INVALID_ARG
+    # the thumbnail form needs bf16 K here: the append writes it
+    assert app_tr(k=None) == ffd.FFD_ERR_INVALID_ARG
+    assert app_tr(vn=None) == ffd.FFD_ERR_INVALID_ARG and app_tr(re=None) == ffd.FFD_ERR_INVALID_ARG
+
+
 def test_product_path_never_touches_the_oracle():
     for dirpath, _, files in os.walk(PKG):
         for f in files:
