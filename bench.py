@@ -422,12 +422,17 @@ def time_gated_decodes(rep, delta, n, device):
 
 
 def e2e_steps(w, inp, device, delta, steps):
-    """End-to-end decode steps through the public API with host buffers: one
-    pinned H2D copy of the step's query and new key/value rows, one fused
-    launch (append into the cache + last-block re-quantisation + decode,
-    ffd_decode_append), D2H of output and mask."""
+    """End-to-end decode steps through the public API with host buffers.
+
+    graph (the reported value): sparse_long_context_ffd_b200.step.DecodeStep,
+    one CUDA-graph launch per step holding the pinned H2D copy of the query
+    and the new key/value rows, the fused append + re-quantisation + decode
+    launch (ffd_decode_append) and the D2H copies of output and mask, then a
+    stream synchronisation.  eager: the same three stages issued from Python
+    each step."""
     import torch
     from sparse_long_context_ffd_b200 import ffd
+    from sparse_long_context_ffd_b200.step import DecodeStep
     shape = ffd.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.capacity, w.block_size,
                            w.split_blocks)
 
@@ -438,47 +443,77 @@ def e2e_steps(w, inp, device, delta, steps):
     v = bf16(inp["v"]).to(device)
     lengths_h = inp["lengths"]
     lengths = torch.from_numpy(np.ascontiguousarray(lengths_h)).to(device)
-    bufs = ffd.DecodeBuffers(shape, device=device)
-    ffd.quantize_keys(shape, k, lengths, 0, bufs.k_packed, bufs.k_scales)
-    B, Hq, Hkv, D = w.batch, w.num_q_heads, w.num_kv_heads, 128
-    # pinned host inputs, one flat buffer: q [B,Hq,D] | k_new [B,Hkv,D] | v_new [B,Hkv,D]
-    nq, nk = B * Hq * D, B * Hkv * D
-    host_in = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
-    host_in[:nq] = bf16(inp["q"]).reshape(-1)
+    B = w.batch
     last = [int(lengths_h[b]) - 1 for b in range(B)]
-    host_in[nq:nq + nk] = torch.stack([bf16(inp["k"][b, :, last[b]]) for b in range(B)]).reshape(-1)
-    host_in[nq + nk:] = torch.stack([bf16(inp["v"][b, :, last[b]]) for b in range(B)]).reshape(-1)
-    dev_in = torch.empty_like(host_in, device=device)
-    q_d = dev_in[:nq].view(B, Hq, D)
-    k_new = dev_in[nq:nq + nk].view(B, Hkv, D)
-    v_new = dev_in[nq + nk:].view(B, Hkv, D)
-    host_out = torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory()
-    host_mask = torch.empty(bufs.mask.shape, dtype=torch.int32).pin_memory()
+    # the step appends each sequence's last token again: every step does the
+    # same work on the same lengths
+    st = DecodeStep(shape, k, v, lengths, delta)
+    st.host_q.copy_(bf16(inp["q"]))
+    st.host_k_new.copy_(torch.stack([bf16(inp["k"][b, :, last[b]]) for b in range(B)]))
+    st.host_v_new.copy_(torch.stack([bf16(inp["v"][b, :, last[b]]) for b in range(B)]))
     stream = torch.cuda.current_stream(device)
 
-    def one():
-        dev_in.copy_(host_in, non_blocking=True)
-        ffd.decode_append(shape, q_d, k_new, v_new, k, v, bufs.k_packed, bufs.k_scales, lengths,
-                          delta, bufs.out, bufs.mask, bufs.workspace)
-        host_out.copy_(bufs.out, non_blocking=True)
-        host_mask.copy_(bufs.mask, non_blocking=True)
+    def eager():
+        st._body()
         stream.synchronize()
 
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        t0 = time.perf_counter()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            fn()
+        end.record()
+        torch.cuda.synchronize(device)
+        return start.elapsed_time(end) / steps, (time.perf_counter() - t0) * 1e3 / steps
+
+    graph_ms, graph_wall = timed(st.step)
+    eager_ms, eager_wall = timed(eager)
+    if st.check():
+        raise RuntimeError("device flags raised in the end-to-end steps")
+    return {"event_ms_per_step": graph_ms, "wall_ms_per_step": graph_wall,
+            "eager_event_ms_per_step": eager_ms, "eager_wall_ms_per_step": eager_wall,
+            "h2d": st.h2d_bytes, "d2h": st.d2h_bytes}
+
+
+def layer_steps(w, inp, device, delta, steps):
+    """The stand-in attention layer (random weights, hidden = Hq x 128): one
+    graph per step with the pinned H2D of x, the q/k/v projections, the FFD
+    append + decode, the output projection and the D2H of y."""
+    import torch
+    from sparse_long_context_ffd_b200 import ffd
+    from sparse_long_context_ffd_b200.step import StandInAttentionLayer
+    shape = ffd.make_shape(w.batch, w.num_q_heads, w.num_kv_heads, w.capacity, w.block_size,
+                           w.split_blocks)
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    k = bf16(inp["k"]).to(device)
+    v = bf16(inp["v"]).to(device)
+    lengths = torch.from_numpy(np.ascontiguousarray(inp["lengths"])).to(device)
+    hidden = w.num_q_heads * 128
+    # every step re-appends at the same position, so each does the same work
+    layer = StandInAttentionLayer(shape, hidden, k, v, lengths, delta, seed=w.seed, advance=False)
+    layer.host_x.copy_(torch.randn((w.batch, hidden)).to(torch.bfloat16))
     for _ in range(3):
-        one()
-    t0 = time.perf_counter()
+        layer.step()
+    torch.cuda.synchronize(device)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record()
     for _ in range(steps):
-        one()
+        layer.step()
     end.record()
     torch.cuda.synchronize(device)
-    wall = time.perf_counter() - t0
-    h2d = host_in.numel() * 2
-    d2h = host_out.numel() * 2 + host_mask.numel() * 4
-    return {"event_ms_per_step": start.elapsed_time(end) / steps, "wall_ms_per_step":
-            wall * 1e3 / steps, "h2d": h2d, "d2h": d2h}
+    if layer.core.check():
+        raise RuntimeError("device flags raised in the layer steps")
+    return {"us_per_step": start.elapsed_time(end) / steps * 1e3, "hidden": hidden,
+            "how": "StandInAttentionLayer: one CUDA graph per step (H2D x, q/k/v GEMMs, "
+                   "ffd_decode_append, output GEMM, D2H y), random bf16 weights"}
 
 
 # ------------------------------------------------------------- CPU oracle --
@@ -756,6 +791,7 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         e2e = e2e_steps(w, inp, device, w.delta, args.e2e_steps)
     e2e_us = dist_max(e2e["event_ms_per_step"] * 1e3, world, device) if e2e else None
+    layer = layer_steps(w, inp, device, w.delta, min(args.e2e_steps, 200)) if e2e else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -799,9 +835,13 @@ def run_gpu(args):
             "e2e": ({"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                      "d2h_bytes_per_step": e2e["d2h"],
                      "wall_ms_per_step": e2e["wall_ms_per_step"],
-                     "how": "public Python API per step: one pinned H2D of q + new K/V rows, "
-                            "decode_append (cache append + last-block re-quantisation + decode "
-                            "in one launch), D2H out+mask, stream sync"} if e2e else None),
+                     "eager_value": e2e["eager_event_ms_per_step"] * 1e3,
+                     "how": "public API per step (step.DecodeStep): one CUDA-graph launch "
+                            "holding the pinned H2D of q + new K/V rows, ffd_decode_append "
+                            "(cache append + last-block re-quantisation + decode, one kernel) "
+                            "and the D2H of out + mask, then a stream sync; eager_value: the "
+                            "same stages issued from Python each step"} if e2e else None),
+            "stand_in_layer": layer,
             "cpu_baseline": cpu,
             "gpu_launches": args.steps,
             "gpu_launches_note": "one fused decode launch per timed step (the headline int4 "

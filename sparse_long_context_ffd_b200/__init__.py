@@ -8,3 +8,4 @@ from . import ffd  # noqa: F401
 from .ffd import (FFDError, Shape, DecodeBuffers, decode, quantize_keys, make_shape,  # noqa: F401
                   workspace_init, decode_workspace_bytes, check_device_status,
                   FFD_LAST_BLOCK)
+from .step import DecodeStep, StandInAttentionLayer  # noqa: F401,E402
