@@ -425,11 +425,11 @@ def e2e_steps(w, inp, device, delta, steps):
     """End-to-end decode steps through the public API with host buffers.
 
     graph (the reported value): sparse_long_context_ffd_b200.step.DecodeStep,
-    one CUDA-graph launch per step holding the pinned H2D copy of the query
-    and the new key/value rows, the fused append + re-quantisation + decode
-    launch (ffd_decode_append) and the D2H copies of output and mask, then a
-    stream synchronisation.  eager: the same three stages issued from Python
-    each step."""
+    one call per step into the library's native step graph: the pinned H2D
+    copy of the query and the new key/value rows, then the fused append +
+    re-quantisation + decode launch (ffd_decode_append), which writes output
+    and mask straight into pinned host memory; the call waits for the graph.
+    eager: H2D, the launch and a D2H copy issued from Python each step."""
     import torch
     from sparse_long_context_ffd_b200 import ffd
     from sparse_long_context_ffd_b200.step import DecodeStep
@@ -836,11 +836,12 @@ def run_gpu(args):
                      "d2h_bytes_per_step": e2e["d2h"],
                      "wall_ms_per_step": e2e["wall_ms_per_step"],
                      "eager_value": e2e["eager_event_ms_per_step"] * 1e3,
-                     "how": "public API per step (step.DecodeStep): one CUDA-graph launch "
-                            "holding the pinned H2D of q + new K/V rows, ffd_decode_append "
-                            "(cache append + last-block re-quantisation + decode, one kernel) "
-                            "and the D2H of out + mask, then a stream sync; eager_value: the "
-                            "same stages issued from Python each step"} if e2e else None),
+                     "how": "public API per step (step.DecodeStep -> ffd_step_graph_run): "
+                            "one native CUDA graph holding the pinned H2D of q + new K/V rows "
+                            "and ffd_decode_append (cache append + last-block re-quantisation + "
+                            "decode, one kernel, writing out + mask straight into pinned host "
+                            "memory), then a stream sync; eager_value: H2D, launch and D2H "
+                            "issued from Python each step"} if e2e else None),
             "stand_in_layer": layer,
             "cpu_baseline": cpu,
             "gpu_launches": args.steps,

@@ -265,6 +265,41 @@ ffd_status ffd_decode_append_tr(const ffd_shape *shape, int32_t reference, const
                                 uint32_t *mask, void *workspace, size_t workspace_bytes,
                                 void *cuda_stream);
 
+/* ---- One layer's whole decode step as a native CUDA graph ----
+ * gist.science explainer, Methodology 3: the decoding step is captured whole in
+ * a CUDA graph, so a small batch pays no CPU launch overhead.  The graph
+ * (captured here on a private stream, nothing is executed at creation) holds:
+ *   1. the H2D copy of host_in -> dev_in, both laid out as
+ *      q bf16 [B][Hq][D] | k_new bf16 [B][Hkv][D] | v_new bf16 [B][Hkv][D]
+ *      (host_in must be pinned host memory);
+ *   2. when advance == 1, lengths[b] += 1 for every sequence;
+ *   3. ffd_decode_append (format 0: k_copy = k_packed, k_resid unused) or
+ *      ffd_decode_append_tr (format 1: k_copy = k_thumb), writing the output
+ *      rows at dev_result and the mask at dev_result + mask_offset (a
+ *      multiple of 16, at least B*Hq*D*2 bytes);
+ *   4. the D2H copy of dev_result (mask_offset + 4 * ffd_mask_words bytes) to
+ *      host_result (pinned).  With dev_result == NULL the kernel writes the
+ *      results straight into host_result, which must then be pinned host
+ *      memory mapped into the device address space (the default for pinned
+ *      memory under unified addressing), and the graph has no D2H node.
+ * ffd_step_graph_run launches it and waits for it on the graph's stream: a
+ * decode step from host inputs to host outputs in one call.  All buffers stay
+ * caller-owned and must outlive the graph; the caller orders its own earlier
+ * device work (cache prefill, quantisation) before the first run, e.g. with a
+ * device synchronisation.  This object is the one place the library keeps
+ * state: a stream, a graph and its executable, released by
+ * ffd_step_graph_destroy.  Argument checks as ffd_decode_append; a failure
+ * returns a status and no graph. */
+typedef struct ffd_step_graph ffd_step_graph;
+ffd_status ffd_step_graph_create(const ffd_shape *shape, int32_t format, int32_t reference,
+                                 float delta, int32_t advance, const void *host_in, void *dev_in,
+                                 void *k_bf16, void *v_bf16, void *k_copy, void *k_resid,
+                                 void *k_scales, int32_t *d_lengths, void *dev_result,
+                                 void *host_result, size_t mask_offset, void *workspace,
+                                 size_t workspace_bytes, ffd_step_graph **graph_out);
+ffd_status ffd_step_graph_run(ffd_step_graph *graph);
+void ffd_step_graph_destroy(ffd_step_graph *graph);
+
 /* Context (sequence) sharding across GPUs.  Each rank holds a contiguous
  * shard of every sequence's cache: rank r holds global tokens
  * [r * cap_local, (r + 1) * cap_local) in a cache of capacity cap_local, with

@@ -1051,26 +1051,43 @@ size_t smem_bytes_tf(int split_blocks) {
          2 * static_cast<size_t>((split_blocks + 7) & ~7);
 }
 
+// Raise the kernel's dynamic shared memory cap once per device, to the
+// largest split this build accepts, so later launches (and graph captures)
+// need no attribute call.
 template <int T, int G, int F>
-cudaError_t launch_tgf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
-                       size_t smem, cudaStream_t stream) {
-  auto kern = decode_kernel<T, G, F>;
-  // Raise the dynamic shared memory cap once per device, to the largest
-  // split this build accepts, so later launches (and graph captures) need
-  // no attribute call.
+cudaError_t configure_tgf() {
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
   if (bit == 0 || (configured.load(std::memory_order_acquire) & bit) == 0) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<T, G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_bytes_tf<T, F>(FFD_MAX_SPLIT_BLOCKS)));
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  kern<<<grid, kThreads, smem, stream>>>(p, tk, tv);
+  return cudaSuccess;
+}
+
+template <int T, int G, int F>
+cudaError_t launch_tgf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
+                       size_t smem, cudaStream_t stream) {
+  cudaError_t e = configure_tgf<T, G, F>();
+  if (e != cudaSuccess) return e;
+  decode_kernel<T, G, F><<<grid, kThreads, smem, stream>>>(p, tk, tv);
   return cudaGetLastError();
+}
+
+template <int T, int F>
+cudaError_t configure_tf(int group) {
+  switch (group) {
+    case 1: return configure_tgf<T, 1, F>();
+    case 2: return configure_tgf<T, 2, F>();
+    case 4: return configure_tgf<T, 4, F>();
+    case 8: return configure_tgf<T, 8, F>();
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int T, int F>
@@ -1102,6 +1119,14 @@ size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format
                             : smem_bytes_tf<128, kFormatThumbResid>(split_blocks);
   return block_size == 64 ? smem_bytes_tf<64, kFormatInt4>(split_blocks)
                           : smem_bytes_tf<128, kFormatInt4>(split_blocks);
+}
+
+cudaError_t prepare_decode(int block_size, int group, int format) {
+  const bool tr = format == kFormatThumbResid;
+  if (block_size == 64) return tr ? configure_tf<64, kFormatThumbResid>(group) : configure_tf<64, kFormatInt4>(group);
+  if (block_size == 128)
+    return tr ? configure_tf<128, kFormatThumbResid>(group) : configure_tf<128, kFormatInt4>(group);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,

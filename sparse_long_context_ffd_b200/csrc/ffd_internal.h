@@ -100,6 +100,11 @@ cudaError_t launch_merge(const MergeParams &p, int block_size, int group, dim3 g
                          cudaStream_t stream);
 cudaError_t launch_quantize(const QuantizeParams &p, int block_size, dim3 grid,
                             cudaStream_t stream);
+// Kernel attributes for a (block size, group, format) variant, set once per
+// device; launch_decode does it too, this lets a caller do it before a graph
+// capture.
+cudaError_t prepare_decode(int block_size, int group, int format);
+
 // tmap_k maps the bf16 K cache (int4 format) or the residuals (thumbnail
 // format); tmap_v the bf16 V cache.
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k,

@@ -36,6 +36,7 @@ EXPORTED = (
     "ffd_decode_ex", "ffd_decode_partials", "ffd_partials_region", "ffd_merge_partials",
     "ffd_thumb_bytes", "ffd_residual_bytes", "ffd_quantize_keys_tr", "ffd_decode_tr",
     "ffd_decode_partials_tr", "ffd_decode_append", "ffd_decode_append_tr",
+    "ffd_step_graph_create", "ffd_step_graph_run", "ffd_step_graph_destroy",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -111,6 +112,14 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_decode_append_tr.argtypes = [sp, i32, p, p, p, p, p, p, p, p, p,
                                                  ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode_append_tr.restype = st
+            lib.ffd_step_graph_create.argtypes = [sp, i32, i32, ctypes.c_float, i32, p, p, p, p,
+                                                  p, p, p, p, p, p, sz, p, sz,
+                                                  ctypes.POINTER(ctypes.c_void_p)]
+            lib.ffd_step_graph_create.restype = st
+            lib.ffd_step_graph_run.argtypes = [p]
+            lib.ffd_step_graph_run.restype = st
+            lib.ffd_step_graph_destroy.argtypes = [p]
+            lib.ffd_step_graph_destroy.restype = None
             lib.ffd_decode.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p, sz, p]
             lib.ffd_decode.restype = st
             lib.ffd_decode_ex.argtypes = [sp, ctypes.POINTER(DecodeOptions), p, p, p, p, p, p,
@@ -385,3 +394,35 @@ class ThumbResidBuffers(DecodeBuffers):
         self.k_packed = None
         self.k_thumb = torch.empty((B, Hkv, cap, D // 4), dtype=torch.uint8, device=device)
         self.k_resid = torch.empty((B, Hkv, cap, D), dtype=torch.uint8, device=device)
+
+
+class StepGraph:
+    """Owner of a native decode-step graph (ffd_step_graph_*): one call runs
+    H2D of the inputs, the fused append + decode and D2H of the results."""
+
+    def __init__(self, shape: Shape, fmt: int, reference: int, delta: float, advance: bool,
+                 host_in, dev_in, k, v, k_copy, k_resid, k_scales, lengths, dev_result,
+                 host_result, mask_offset: int, workspace):
+        self._lib = load_library()
+        handle = ctypes.c_void_p(None)
+        _check(self._lib.ffd_step_graph_create(
+            ctypes.byref(shape), int(fmt), int(reference), float(delta), 1 if advance else 0,
+            host_in.data_ptr(), _ptr(dev_in), _ptr(k), _ptr(v), _ptr(k_copy), _ptr(k_resid),
+            _ptr(k_scales), _ptr(lengths), _ptr(dev_result), host_result.data_ptr(),
+            int(mask_offset), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            ctypes.byref(handle)), "ffd_step_graph_create")
+        self._handle = handle
+
+    def run(self) -> None:
+        _check(self._lib.ffd_step_graph_run(self._handle), "ffd_step_graph_run")
+
+    def close(self) -> None:
+        if self._handle is not None and self._handle.value:
+            self._lib.ffd_step_graph_destroy(self._handle)
+        self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown
+            pass

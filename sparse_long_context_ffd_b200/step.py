@@ -5,11 +5,13 @@ and System Optimization": the entire decoding step is captured in a CUDA graph
 to remove CPU launch overhead at small batch) applied to the FFD step:
 
 * :class:`DecodeStep` -- one layer's FFD decode with host-side inputs and
-  outputs.  The graph holds the H2D copy of the step's query and new K/V rows
-  from pinned memory, optionally the length increment, the fused append +
-  re-quantisation + decode launch (``ffd_decode_append``), and the D2H copies
-  of the output rows and the mask.  A step is one graph launch and one stream
-  synchronisation.
+  outputs, as the library's native step graph (``ffd_step_graph_*``): the H2D
+  copy of the step's query and new K/V rows from pinned memory, optionally the
+  length increment, and the fused append + re-quantisation + decode launch
+  (``ffd_decode_append``), whose kernel writes the output rows and the mask
+  straight into pinned host memory (or, with ``results_to_host`` off, one D2H
+  copy does).  A step is one call into the library, which launches the graph
+  and waits.
 * :class:`StandInAttentionLayer` -- a decode-step attention layer with random
   weights (there is no checkpoint): q, k and v projections of the hidden
   state, the FFD step, the output projection, captured whole.  The
@@ -54,11 +56,14 @@ class DecodeStep:
 
     def __init__(self, shape: ffd.Shape, k_cache, v_cache, lengths, delta: float,
                  reference: int = ffd.FFD_REFERENCE_RUNNING_MAX, fmt: str = "int4",
-                 advance: bool = False):
+                 advance: bool = False, results_to_host: bool = True):
         torch = _require_torch()
         if fmt not in ("int4", "tr"):
             raise ValueError("fmt must be 'int4' or 'tr'")
         self.torch, self.shape, self.fmt = torch, shape, fmt
+        # the graph's kernel writes output and mask straight into pinned host
+        # memory (no D2H copy) unless results_to_host is off
+        self.results_to_host = bool(results_to_host)
         self.delta, self.reference, self.advance = float(delta), int(reference), bool(advance)
         self.k, self.v, self.lengths = k_cache, v_cache, lengths
         dev = k_cache.device
@@ -84,6 +89,7 @@ class DecodeStep:
         out_bytes = B * Hq * D * 2
         mask_off = (out_bytes + 15) // 16 * 16
         total = mask_off + (mask_shape[0] * mask_shape[1] * mask_shape[2]) * 4
+        self._mask_off = mask_off
         self._dev_res = torch.empty(total, dtype=torch.uint8, device=dev)
         self._host_res = torch.empty(total, dtype=torch.uint8).pin_memory()
         b.out = self._dev_res[:out_bytes].view(torch.bfloat16).view(B, Hq, D)
@@ -114,30 +120,24 @@ class DecodeStep:
         self._host_res.copy_(self._dev_res, non_blocking=True)
 
     def capture(self):
-        """Record the step into a CUDA graph (done by the first :meth:`step`).
-        The step first runs once eagerly on the capture stream with the current
-        host inputs, so fill them before capturing; with ``advance`` set that
-        run's length increment is undone (its append is repeated by the replay)."""
-        torch = self.torch
-        saved = self.lengths.clone() if self.advance else None
-        with torch.cuda.stream(self._stream):
-            self._body()  # warm-up outside the graph (loads the library, tensor maps)
-        self._stream.synchronize()
-        if saved is not None:
-            self.lengths.copy_(saved)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=self._stream):
-            self._body()
-        self._graph = g
-        torch.cuda.synchronize(self.k.device)
-        return g
+        """Build the native step graph (done by the first :meth:`step`).
+        Nothing runs at capture; earlier device work on the caches is ordered
+        first by a device synchronisation."""
+        self.torch.cuda.synchronize(self.k.device)
+        b = self.bufs
+        tr = self.fmt == "tr"
+        self._graph = ffd.StepGraph(
+            self.shape, 1 if tr else 0, self.reference, self.delta, self.advance, self._host_in,
+            self._dev_in, self.k, self.v, b.k_thumb if tr else b.k_packed, b.k_resid if tr else None,
+            b.k_scales, self.lengths, None if self.results_to_host else self._dev_res,
+            self._host_res, self._mask_off, b.workspace)
+        return self._graph
 
     def step(self):
-        """One decode step: replay the graph and wait for its D2H copies."""
+        """One decode step: host inputs -> host outputs (one library call)."""
         if self._graph is None:
             self.capture()
-        self._graph.replay()
-        self.torch.cuda.current_stream(self.k.device).synchronize()
+        self._graph.run()
 
     def check(self) -> int:
         """Device flags (ffd.FFD_DEVICE_FLAG_*) raised since the last check."""
