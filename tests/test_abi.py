@@ -190,6 +190,32 @@ def test_append_arguments_rejected_on_host():
     assert app_tr(vn=None) == ffd.FFD_ERR_INVALID_ARG and app_tr(re=None) == ffd.FFD_ERR_INVALID_ARG
 
 
+def test_step_graph_rejects_bad_arguments_without_capturing():
+    lib = ffd.load_library()
+    s = ffd.make_shape(2, 16, 4, 4096, 64, 16)
+    a = 1 << 20
+    out = ctypes.c_void_p(None)
+
+    def create(fmt=0, adv=0, hin=a, din=a, hres=a, mask_off=16384, shape=s, res_ptr=None):
+        return lib.ffd_step_graph_create(ctypes.byref(shape), fmt, 0, 1.0, adv, hin, din, a, a, a,
+                                         a, a, a, res_ptr, hres, mask_off, a, 1 << 30,
+                                         ctypes.byref(out))
+
+    assert lib.ffd_step_graph_create(ctypes.byref(s), 0, 0, 1.0, 0, a, a, a, a, a, a, a, a, a, a,
+                                     16384, a, 1 << 30, None) == ffd.FFD_ERR_INVALID_ARG
+    assert create(fmt=2) == ffd.FFD_ERR_INVALID_ARG
+    assert create(adv=3) == ffd.FFD_ERR_INVALID_ARG
+    assert create(hin=None) == ffd.FFD_ERR_INVALID_ARG
+    assert create(din=a + 8) == ffd.FFD_ERR_INVALID_ARG
+    assert create(hres=a + 4) == ffd.FFD_ERR_INVALID_ARG
+    assert create(mask_off=100) == ffd.FFD_ERR_INVALID_ARG      # not a multiple of 16
+    assert create(mask_off=16) == ffd.FFD_ERR_INVALID_ARG       # inside the output rows
+    assert create(shape=ffd.make_shape(0, 16, 4, 4096, 64, 16)) == ffd.FFD_ERR_INVALID_ARG
+    assert out.value is None
+    lib.ffd_step_graph_destroy(None)  # a null graph is ignored
+    assert lib.ffd_step_graph_run(None) == ffd.FFD_ERR_INVALID_ARG
+
+
 def test_product_path_never_touches_the_oracle():
     for dirpath, _, files in os.walk(PKG):
         for f in files:
