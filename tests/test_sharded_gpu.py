@@ -54,6 +54,45 @@ def test_sharded_decode_matches_unsharded(W, T, S, G, delta):
     assert_output_close(bf16_to_np_f32(out).astype(np.float64), want_out, f"W{W} delta {delta}")
 
 
+@pytest.mark.parametrize("W,T,S", [(2, 64, 4), (3, 128, 2)])
+@pytest.mark.parametrize("delta", [1.0, float("inf")])
+def test_sharded_thumb_resid_decode_matches_unsharded(W, T, S, delta):
+    # the same exchange on the 2-bit thumbnail + 8-bit residual key format
+    cap_local = T * S * 4
+    cap = W * cap_local
+    B, Hkv, G = 3, 2, 4
+    w = fw.random_small_workload(97 + W, B, G, Hkv, cap, T, S, delta, 1, cap, needles=2)
+    inp = fw.make_inputs(w)
+    lengths = inp["lengths"].copy()
+    lengths[1] = cap_local // 3
+    inp = fw.make_inputs(w, lengths=lengths)
+    thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], lengths, T)
+    want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales, lengths, T,
+                                              S, delta)
+    local = ffd.make_shape(B, G * Hkv, Hkv, cap_local, T, S)
+    q = to_dev_bf16(inp["q"])
+    off, nbytes = ffd.partials_region(local)
+    regions = []
+    for r in range(W):
+        sl = slice(r * cap_local, (r + 1) * cap_local)
+        k_r = to_dev_bf16(np.ascontiguousarray(inp["k"][:, :, sl]))
+        v_r = to_dev_bf16(np.ascontiguousarray(inp["v"][:, :, sl]))
+        ln_r = torch.from_numpy(sharded.local_lengths(lengths, r, cap_local)).cuda()
+        bufs = ffd.ThumbResidBuffers(local)
+        ffd.quantize_keys_tr(local, k_r, ln_r, 0, bufs.k_thumb, bufs.k_resid, bufs.k_scales)
+        ffd.decode_partials_tr(local, q, k_r, v_r, bufs.k_thumb, bufs.k_resid, bufs.k_scales, ln_r,
+                               delta, bufs.workspace, requant_last=(r == 0))
+        regions.append(bufs.workspace[off:off + nbytes].clone())
+        assert ffd.check_device_status(bufs.workspace) == 0
+    out = torch.full((B, G * Hkv, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    mask = torch.full((B, Hkv, sharded.global_mask_words(W, cap_local, T)), -1, dtype=torch.int32,
+                      device="cuda")
+    ffd.merge_partials(local, W, torch.cat(regions), torch.from_numpy(lengths).cuda(), out, mask)
+    torch.cuda.synchronize()
+    assert_mask_equal(mask.cpu().numpy().view(np.uint32), want_mask, f"tr W{W} delta {delta}")
+    assert_output_close(bf16_to_np_f32(out).astype(np.float64), want_out, f"tr W{W} delta {delta}")
+
+
 def test_sharded_entry_points_reject_bad_shapes():
     import ctypes
     lib = ffd.load_library()
