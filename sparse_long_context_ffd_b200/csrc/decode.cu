@@ -43,6 +43,7 @@ namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr float kRsqrtD = 0.08838834764831845f;     // nearest float to 1/sqrt(128)
+constexpr float kFltMax = 3.4028234663852886e38f;
 constexpr float kScaleLog2 = 0.12751743074195287f;  // log2(e) / sqrt(128)
 
 // Pipeline geometry.
@@ -157,183 +158,191 @@ __device__ __forceinline__ int scan_block_index(int e, int nref, int nb, int j0)
   return e < nref ? (e == 0 ? 0 : nb - 1) : j0 + (e - nref);
 }
 
-// Selector for one block (executed by one warp): fold the group's query with
-// the block's channel scales into int8, integer-score every token on the
-// tensor cores and return, in lane (0, t4), the scores of heads 2*t4 and
-// 2*t4 + 1.
+// Query fold of the selector (the per-block int8 query: p_c = q_c s_c,
+// a = max |p_c|, qi_c = rint(p_c 127 / a)), spread over the warp.  Lane
+// (gid, t4) folds head gid % G over part r = gid / G of the 32 channels
+// 32*t4 .. 32*t4 + 31 that its mma B fragments cover, R parts per head so
+// that every lane group works when G < 8; the int8 words are then gathered
+// into the B fragments of lanes gid < G (lanes gid >= G feed output columns
+// of heads that do not exist, so their fragments are left as they fall).
 //
-// Lane (gid = lane / 4, t4 = lane % 4) folds head gid over channels
-// 32*t4 .. 32*t4 + 31, which are exactly the channels its mma B fragments
-// hold: k-step s takes packed word s of the lane's 16-byte chunk of a token
-// row, whose low nibbles are channels 32*t4 + 8s + {0,2,4,6} and high
-// nibbles channels 32*t4 + 8s + {1,3,5,7}.
-template <int T, int G>
-__device__ __forceinline__ void scan_block(const uint8_t *tile, const uint16_t *scl,
-                                           const uint32_t (&qreg)[16], int valid_rows, int lane,
-                                           float &score0, float &score1) {
-  const int gid = lane >> 2, t4 = lane & 3;
-  float pc[32];
-  float a = 0.0f;
-  const uint4 *s4 = reinterpret_cast<const uint4 *>(scl) + 4 * t4;
-#pragma unroll
-  for (int w4 = 0; w4 < 4; ++w4) {
-    const uint4 sv = s4[w4];
-    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = 8 * w4 + 2 * e;
-      const uint32_t qw = qreg[k >> 1];
-      pc[k] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
-      pc[k + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
-      a = fmaxf(a, fmaxf(fabsf(pc[k]), fabsf(pc[k + 1])));
-    }
+// B word positions pos = 0..7 (the order of the fragment registers):
+//   int4 format   pos = 2s + x: k-step s, x = 0 for the low nibbles
+//                 (channels 8s + {0,2,4,6}), 1 for the high ones (+1);
+//   thumbnail     pos = 4h + k: k-step k, word group h, bytes channels
+//                 16h + {2k, 8+2k, 2k+1, 9+2k}.
+// Part r owns positions r*NW .. r*NW + NW - 1.  Its channels are
+// base(r) + off(ci), ci = 0..NC-1 (the lane's compact order), and byte j of
+// its word w is compact index idx(w, j).
+template <int G, int F>
+struct ScanFold {
+  static constexpr bool kTR = F == kFormatThumbResid;
+  static constexpr int R = G >= 8 ? 1 : (G == 4 ? 2 : 4);
+  static constexpr int NC = 32 / R;  // channels folded per lane
+  static constexpr int NW = NC / 4;  // int8 B words per lane
+  // the thumbnail format with 4 parts takes channels base + {0..3, 8..11}
+  static constexpr bool kSplitRuns = kTR && R == 4;
+  __device__ static int part(int gid) { return (gid / G) & (R - 1); }
+  __device__ static int base(int r) { return kSplitRuns ? 16 * (r >> 1) + 4 * (r & 1) : r * NC; }
+  static constexpr int off(int ci) { return kSplitRuns && ci >= 4 ? ci + 4 : ci; }
+  static constexpr int idx(int w, int j) {
+    if (!kTR) return 8 * (w >> 1) + 2 * j + (w & 1);
+    if (kSplitRuns) return j == 0 ? 2 * w : j == 1 ? 4 + 2 * w : j == 2 ? 2 * w + 1 : 5 + 2 * w;
+    const int k = w & 3, h16 = 16 * (w >> 2);
+    return h16 + (j == 0 ? 2 * k : j == 1 ? 8 + 2 * k : j == 2 ? 2 * k + 1 : 9 + 2 * k);
   }
-  a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
-  a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
-
-  uint32_t bq[4][2];
-  int sumq = 0;
-  float cf = 0.0f;
-  if (gid < G && a > 0.0f) {
-    const float inv = __fdiv_rn(127.0f, a);
+  // the lane's NC bf16 values of a channel row (query or scales) as pairs
+  template <typename Src>
+  __device__ static void load_pairs(const Src *row_t4, int r, uint32_t (&v)[NC / 2]) {
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(row_t4) + base(r);
+    if constexpr (kSplitRuns) {
+      const uint2 x = *reinterpret_cast<const uint2 *>(src);
+      const uint2 y = *reinterpret_cast<const uint2 *>(src + 8);
+      v[0] = x.x;
+      v[1] = x.y;
+      v[2] = y.x;
+      v[3] = y.y;
+    } else {
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int ql = clamp127(__float2int_rn(__fmul_rn(pc[8 * s + 2 * e], inv)));
-        const int qh = clamp127(__float2int_rn(__fmul_rn(pc[8 * s + 2 * e + 1], inv)));
-        sumq += ql + qh;
-        lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * e);
-        hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * e);
+      for (int m = 0; m < NC / 8; ++m) {
+        const uint4 x = reinterpret_cast<const uint4 *>(src)[m];
+        v[4 * m] = x.x;
+        v[4 * m + 1] = x.y;
+        v[4 * m + 2] = x.z;
+        v[4 * m + 3] = x.w;
       }
-      bq[s][0] = lo;
-      bq[s][1] = hi;
     }
-    cf = __fmul_rn(__fdiv_rn(a, 127.0f), kRsqrtD);
-  } else {
-#pragma unroll
-    for (int s = 0; s < 4; ++s) bq[s][0] = bq[s][1] = 0u;
   }
-  sumq += __shfl_xor_sync(kFull, sumq, 1);
-  sumq += __shfl_xor_sync(kFull, sumq, 2);
+};
 
-  // sum_c qi_c * (u_c - 8) = sum_c qi_c * u_c - 8 * sum_c qi_c, and the
-  // correction commutes with the max over tokens.
-  int best0 = INT_MIN, best1 = INT_MIN;  // heads 2*t4, 2*t4 + 1
-#pragma unroll
-  for (int mt = 0; mt < T / 16; ++mt) {
-    const int r0 = 16 * mt + gid, r1 = r0 + 8;
-    const uint4 u0 = *reinterpret_cast<const uint4 *>(tile + r0 * kPackedRowBytes + 16 * t4);
-    const uint4 u1 = *reinterpret_cast<const uint4 *>(tile + r1 * kPackedRowBytes + 16 * t4);
-    const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w};
-    const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w};
-    int acc[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      mma_u8s8_16x8x32(acc, w0[s] & 0x0F0F0F0Fu, w1[s] & 0x0F0F0F0Fu, (w0[s] >> 4) & 0x0F0F0F0Fu,
-                       (w1[s] >> 4) & 0x0F0F0F0Fu, bq[s][0], bq[s][1]);
-    }
-    if (r0 < valid_rows) {
-      best0 = max(best0, acc[0]);
-      best1 = max(best1, acc[1]);
-    }
-    if (r1 < valid_rows) {
-      best0 = max(best0, acc[2]);
-      best1 = max(best1, acc[3]);
-    }
-  }
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    best0 = max(best0, __shfl_xor_sync(kFull, best0, off));
-    best1 = max(best1, __shfl_xor_sync(kFull, best1, off));
-  }
-  const int h0 = 2 * t4, h1 = 2 * t4 + 1;
-  const int sq0 = __shfl_sync(kFull, sumq, h0 << 2);
-  const int sq1 = __shfl_sync(kFull, sumq, h1 << 2);
-  const float c0 = __shfl_sync(kFull, cf, h0 << 2);
-  const float c1 = __shfl_sync(kFull, cf, h1 << 2);
-  score0 = __fmul_rn(__int2float_rn(best0 - 8 * sq0), c0);
-  score1 = __fmul_rn(__int2float_rn(best1 - 8 * sq1), c1);
+// Low byte of four words packed into one (bytes 0..3 from a, b, c, d).
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
 
-// Selector for one block of 2-bit thumbnails (same contract as scan_block).
-// The fold is the int4 one; the thumbnail level of code u is (2u - 3) s / 2,
-// so I_t = sum_c qi_c (2 u_c - 3) = 2 sum_c qi_c u_c - 3 sum_c qi_c and the
-// score is float(max_t I_t) * (a / 254) / sqrt(D).
+// Fold one block's scales into the int8 query (see ScanFold).  qv: the lane's
+// query channels in compact order, as bf16 pairs.  Returns the B fragments in bq
+// (lanes gid < G), the head's sum of qi in sumq and a in a_out (every lane of
+// the head; a == 0 gives qi = 0).
 //
-// Lane (gid, t4) again owns channels 32*t4 .. 32*t4 + 31 = thumbnail words
-// 2*t4 and 2*t4 + 1 of a token row.  (w >> 2k) & 0x03030303 puts channels
-// 16w' + {2k, 8+2k, 2k+1, 9+2k} (w' the word's group) in bytes 0..3, so
-// k-step k takes a0 from word 2*t4 and a2 from word 2*t4 + 1, and the int8
-// query is packed in the same channel order.
-template <int T, int G>
-__device__ __forceinline__ void scan_block_tr(const uint8_t *tile, const uint16_t *scl,
-                                              const uint32_t (&qreg)[16], int valid_rows, int lane,
-                                              float &score0, float &score1) {
+// Rounding: with the fp32 product x = p * (127 / a), |x| <= 127 (1 + 2^-24)^2
+// < 127.5, so the fp32 sum x + 1.5 * 2^23 is 1.5 * 2^23 + rint(x) exactly
+// (round to nearest even, as rint), its low byte is qi as int8 and the clamp
+// to +-127 never acts.  When 127 / a overflows (a below about 3.7e-37), or a
+// itself is infinite, the conversion is done the direct way instead.
+template <int G, int F>
+__device__ __forceinline__ void fold_block(const uint16_t *scl, const uint32_t (&qv)[ScanFold<G, F>::NC / 2],
+                                           int lane, uint32_t (&bq)[8], int &sumq, float &a_out) {
+  using SF = ScanFold<G, F>;
+  constexpr int NC = SF::NC, NW = SF::NW, R = SF::R;
   const int gid = lane >> 2, t4 = lane & 3;
-  float pc[32];
-  float a = 0.0f;
-  const uint4 *s4 = reinterpret_cast<const uint4 *>(scl) + 4 * t4;
+  const int r = SF::part(gid);
+  uint32_t sv[NC / 2];
+  SF::load_pairs(scl + 32 * t4, r, sv);
+  // p_c is recomputed where it is used (an exact product) rather than kept
+  auto pc = [&](int c) {
+    return (c & 1) ? __fmul_rn(bf16_hi(qv[c >> 1]), bf16_hi(sv[c >> 1])) : __fmul_rn(bf16_lo(qv[c >> 1]), bf16_lo(sv[c >> 1]));
+  };
+  float am0 = 0.0f, am1 = 0.0f;
 #pragma unroll
-  for (int w4 = 0; w4 < 4; ++w4) {
-    const uint4 sv = s4[w4];
-    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int k = 8 * w4 + 2 * e;
-      const uint32_t qw = qreg[k >> 1];
-      pc[k] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
-      pc[k + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
-      a = fmaxf(a, fmaxf(fabsf(pc[k]), fabsf(pc[k + 1])));
-    }
+  for (int c = 0; c < NC; c += 2) {
+    am0 = fmaxf(am0, fabsf(pc(c)));
+    am1 = fmaxf(am1, fabsf(pc(c + 1)));
   }
+  float a = fmaxf(am0, am1);
   a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
   a = fmaxf(a, __shfl_xor_sync(kFull, a, 2));
-
-  uint32_t bq[4][2];
-  int sumq = 0;
-  float cf = 0.0f;
-  if (gid < G && a > 0.0f) {
+#pragma unroll
+  for (int m = 1; m < R; m <<= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, 4 * G * m));
+  uint32_t words[NW];
+  int sq = 0;
+  if (a > 0.0f) {
     const float inv = __fdiv_rn(127.0f, a);
-    int qi[32];
+    if (a <= kFltMax && inv <= kFltMax) {
+      uint32_t acc = 0u;
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      qi[c] = clamp127(__float2int_rn(__fmul_rn(pc[c], inv)));
-      sumq += qi[c];
-    }
-    // k-step k, half h (a0: word 2*t4, a2: word 2*t4 + 1): local channels
-    // 16h + {2k, 8+2k, 2k+1, 9+2k} in bytes 0..3
+      for (int w = 0; w < NW; ++w) {
+        uint32_t y[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+        for (int j = 0; j < 4; ++j) {
+          y[j] = __float_as_uint(__fadd_rn(__fmul_rn(pc(SF::idx(w, j)), inv), 12582912.0f));
+          acc += y[j];
+        }
+        words[w] = low_bytes4(y[0], y[1], y[2], y[3]);
+      }
+      sq = static_cast<int>(acc - static_cast<uint32_t>(NC) * 0x4B400000u);
+    } else {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int c0 = 16 * h + 2 * k;
-        bq[k][h] = (static_cast<uint32_t>(qi[c0]) & 0xFFu) | ((static_cast<uint32_t>(qi[c0 + 8]) & 0xFFu) << 8) |
-                   ((static_cast<uint32_t>(qi[c0 + 1]) & 0xFFu) << 16) |
-                   ((static_cast<uint32_t>(qi[c0 + 9]) & 0xFFu) << 24);
+      for (int w = 0; w < NW; ++w) {
+        uint32_t y[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int v = clamp127(__float2int_rn(__fmul_rn(pc(SF::idx(w, j)), inv)));
+          sq += v;
+          y[j] = static_cast<uint32_t>(v);
+        }
+        words[w] = low_bytes4(y[0], y[1], y[2], y[3]);
       }
     }
-    cf = __fmul_rn(__fdiv_rn(a, 254.0f), kRsqrtD);
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) bq[k][0] = bq[k][1] = 0u;
+    for (int w = 0; w < NW; ++w) words[w] = 0u;
   }
-  sumq += __shfl_xor_sync(kFull, sumq, 1);
-  sumq += __shfl_xor_sync(kFull, sumq, 2);
+  sq += __shfl_xor_sync(kFull, sq, 1);
+  sq += __shfl_xor_sync(kFull, sq, 2);
+#pragma unroll
+  for (int m = 1; m < R; m <<= 1) sq += __shfl_xor_sync(kFull, sq, 4 * G * m);
+  // gather: position pos comes from part pos / NW, NW words on
+#pragma unroll
+  for (int pos = 0; pos < 8; ++pos) {
+    if (pos < NW)
+      bq[pos] = words[pos];
+    else
+      bq[pos] = __shfl_sync(kFull, words[pos % NW], (lane + 4 * G * (pos / NW)) & 31);
+  }
+  sumq = sq;
+  a_out = a;
+}
 
-  int best0 = INT_MIN, best1 = INT_MIN;  // max_t sum_c qi_c u_c, heads 2*t4, 2*t4 + 1
+// Selector, tensor-core part: the integer score sum_c qi_c u_c of every token
+// of a block, maxed over the valid tokens, for heads 2*t4 and 2*t4 + 1 of the
+// lane's output columns (reduced over the warp at the end).
+//
+// int4 format: k-step s takes packed word s of the lane's 16-byte chunk of a
+// token row (channels 32*t4 + 8s .. +7), whose low nibbles are channels
+// 8s + {0,2,4,6} and high nibbles 8s + {1,3,5,7}: B positions 2s and 2s + 1.
+// Thumbnail format: the lane reads thumbnail words 2*t4 + h (h = 0, 1) of its
+// token rows; (w >> 2k) & 0x03030303 puts channels 16h + {2k, 8+2k, 2k+1,
+// 9+2k} (relative to 32*t4) in bytes 0..3, so k-step k takes a0 from word
+// 2*t4 and a2 from word 2*t4 + 1, with B positions k and 4 + k.
+template <int T, int F>
+__device__ __forceinline__ void block_best(const uint8_t *tile, const uint32_t (&bq)[8], int valid_rows,
+                                           int lane, int &best0, int &best1) {
+  const int gid = lane >> 2, t4 = lane & 3;
+  best0 = INT_MIN;
+  best1 = INT_MIN;
 #pragma unroll
   for (int mt = 0; mt < T / 16; ++mt) {
     const int r0 = 16 * mt + gid, r1 = r0 + 8;
-    const uint2 u0 = *reinterpret_cast<const uint2 *>(tile + r0 * kThumbRowBytes + 8 * t4);
-    const uint2 u1 = *reinterpret_cast<const uint2 *>(tile + r1 * kThumbRowBytes + 8 * t4);
     int acc[4] = {0, 0, 0, 0};
+    if constexpr (F == kFormatThumbResid) {
+      const uint2 u0 = *reinterpret_cast<const uint2 *>(tile + r0 * kThumbRowBytes + 8 * t4);
+      const uint2 u1 = *reinterpret_cast<const uint2 *>(tile + r1 * kThumbRowBytes + 8 * t4);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      mma_u8s8_16x8x32(acc, (u0.x >> (2 * k)) & 0x03030303u, (u1.x >> (2 * k)) & 0x03030303u,
-                       (u0.y >> (2 * k)) & 0x03030303u, (u1.y >> (2 * k)) & 0x03030303u, bq[k][0],
-                       bq[k][1]);
+      for (int k = 0; k < 4; ++k) {
+        mma_u8s8_16x8x32(acc, (u0.x >> (2 * k)) & 0x03030303u, (u1.x >> (2 * k)) & 0x03030303u,
+                         (u0.y >> (2 * k)) & 0x03030303u, (u1.y >> (2 * k)) & 0x03030303u, bq[k], bq[4 + k]);
+      }
+    } else {
+      const uint4 u0 = *reinterpret_cast<const uint4 *>(tile + r0 * kPackedRowBytes + 16 * t4);
+      const uint4 u1 = *reinterpret_cast<const uint4 *>(tile + r1 * kPackedRowBytes + 16 * t4);
+      const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w};
+      const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        mma_u8s8_16x8x32(acc, w0[s] & 0x0F0F0F0Fu, w1[s] & 0x0F0F0F0Fu, (w0[s] >> 4) & 0x0F0F0F0Fu,
+                         (w1[s] >> 4) & 0x0F0F0F0Fu, bq[2 * s], bq[2 * s + 1]);
+      }
     }
     if (r0 < valid_rows) {
       best0 = max(best0, acc[0]);
@@ -344,6 +353,21 @@ __device__ __forceinline__ void scan_block_tr(const uint8_t *tile, const uint16_
       best1 = max(best1, acc[3]);
     }
   }
+}
+
+// Selector, last part: the block scores of heads 2*t4 and 2*t4 + 1 from the
+// per-lane maxima, the head's sum of qi and a (every lane).
+//   int4 format:  I = sum_c qi_c (u_c - 8) = sum qi u - 8 sum qi (the
+//                 correction commutes with the max over tokens), score =
+//                 float(max_t I_t) * (a / 127) / sqrt(D);
+//   thumbnails:   the level of code u is (2u - 3) s / 2, so I = 2 sum qi u -
+//                 3 sum qi and score = float(max_t I_t) * (a / 254) / sqrt(D).
+template <int F>
+__device__ __forceinline__ void block_scores(int best0, int best1, int sumq, float a, int lane, float &score0,
+                                             float &score1) {
+  constexpr bool kTR = F == kFormatThumbResid;
+  const int t4 = lane & 3;
+  const float cf = a > 0.0f ? __fmul_rn(__fdiv_rn(a, kTR ? 254.0f : 127.0f), kRsqrtD) : 0.0f;
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     best0 = max(best0, __shfl_xor_sync(kFull, best0, off));
@@ -354,8 +378,13 @@ __device__ __forceinline__ void scan_block_tr(const uint8_t *tile, const uint16_
   const int sq1 = __shfl_sync(kFull, sumq, h1 << 2);
   const float c0 = __shfl_sync(kFull, cf, h0 << 2);
   const float c1 = __shfl_sync(kFull, cf, h1 << 2);
-  score0 = __fmul_rn(__int2float_rn(2 * best0 - 3 * sq0), c0);
-  score1 = __fmul_rn(__int2float_rn(2 * best1 - 3 * sq1), c1);
+  if constexpr (kTR) {
+    score0 = __fmul_rn(__int2float_rn(2 * best0 - 3 * sq0), c0);
+    score1 = __fmul_rn(__int2float_rn(2 * best1 - 3 * sq1), c1);
+  } else {
+    score0 = __fmul_rn(__int2float_rn(best0 - 8 * sq0), c0);
+    score1 = __fmul_rn(__int2float_rn(best1 - 8 * sq1), c1);
+  }
 }
 
 template <int T, int G, int F>
@@ -570,46 +599,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ============================================================ scan warp
   if (warp == kScanWarp) {
     if (dense) return;
+    using SF = ScanFold<G, F>;
     const int gid = lane >> 2, t4 = lane & 3;
-    uint32_t qreg[16];
-    if (gid < G) {
-      const uint4 *qsrc = reinterpret_cast<const uint4 *>(
-          p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid) * kHeadDim +
-          32 * t4);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 x = qsrc[v];
-        qreg[4 * v] = x.x;
-        qreg[4 * v + 1] = x.y;
-        qreg[4 * v + 2] = x.z;
-        qreg[4 * v + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int v = 0; v < 16; ++v) qreg[v] = 0u;
-    }
+    // the lane's query channels in its fold order (see ScanFold)
+    uint32_t qv[SF::NC / 2];
+    SF::load_pairs(p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid % G) *
+                             kHeadDim + 32 * t4,
+                   SF::part(gid), qv);
     float run0 = -INFINITY, run1 = -INFINITY;  // running max of heads 2*t4, 2*t4 + 1
     int qn = 0;
-    for (int e = 0; e < nref + nbs; ++e) {
-      const int st = e % NSA;
-      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, kWaitLimitNs)) {
-        raise_timeout(p, ctrl);
-        break;
-      }
-      const int jb = scan_block_index(e, nref, nb, j0);
-      const uint8_t *tile = scan_ring + st * SG::kStageBytes;
-      float s0, s1;
-      const uint16_t *scl = reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes);
-      if constexpr (kTR)
-        scan_block_tr<T, G>(tile, scl, qreg, min(T, len - jb * T), lane, s0, s1);
-      else
-        scan_block<T, G>(tile, scl, qreg, min(T, len - jb * T), lane, s0, s1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_a[st]);
+    // the Top-delta decision for scan entry e
+    auto decide = [&](int e, float s0, float s1) {
       if (e < nref) {  // reference blocks: the split's running max starts at their max
         run0 = fmaxf(run0, s0);
         run1 = fmaxf(run1, s1);
-        continue;
+        return;
       }
       const int i = e - nref;
       // Top-delta against the running maximum of the split, union over the group
@@ -633,6 +637,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         ++qn;
       }
+    };
+    for (int e = 0; e < nref + nbs; ++e) {
+      const int st = e % NSA;
+      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, kWaitLimitNs)) {
+        raise_timeout(p, ctrl);
+        break;
+      }
+      const int jb = scan_block_index(e, nref, nb, j0);
+      const uint8_t *tile = scan_ring + st * SG::kStageBytes;
+      uint32_t bq[8];
+      int sq, best0, best1;
+      float am, s0, s1;
+      fold_block<G, F>(reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes), qv, lane, bq, sq, am);
+      block_best<T, F>(tile, bq, min(T, len - jb * T), lane, best0, best1);
+      block_scores<F>(best0, best1, sq, am, lane, s0, s1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_a[st]);
+      decide(e, s0, s1);
       if (ctrl[3]) break;
     }
     if (lane == 0) {
@@ -878,12 +900,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     l_run[0] = l_run[0] * corr0 + ps0;
     l_run[1] = l_run[1] * corr1 + ps1;
+    // (the factor is exactly 1 whenever the running max stayed, which is most
+    // stages once it has settled; skipping the multiply changes no bit)
+    if (__any_sync(kFull, corr0 != 1.0f || corr1 != 1.0f)) {
 #pragma unroll
-    for (int cm = 0; cm < 8; ++cm) {
-      oacc[cm][0] *= corr0;
-      oacc[cm][1] *= corr1;
-      oacc[cm][2] *= corr0;
-      oacc[cm][3] *= corr1;
+      for (int cm = 0; cm < 8; ++cm) {
+        oacc[cm][0] *= corr0;
+        oacc[cm][1] *= corr1;
+        oacc[cm][2] *= corr0;
+        oacc[cm][3] *= corr1;
+      }
     }
     // O^T += V^T P^T: 8 channel tiles x kKvTok/16 token steps
 #pragma unroll
