@@ -526,9 +526,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         progress = true;
       }
       // K/V stages for the kept blocks published so far
-      const bool sel_done = dense || ctrl[1] != 0;
-      __threadfence_block();
-      const int avail = dense ? nbs : ctrl[0];
+      // (acquire loads: the queue entries below are read after the count)
+      const bool sel_done = dense || ld_acquire_cta(&ctrl[1]) != 0;
+      const int avail = dense ? nbs : ld_acquire_cta(&ctrl[0]);
       while (q_ptr < avail) {
         const int j = dense ? q_ptr : static_cast<int>(queue[q_ptr]);
         const int tok = (j0 + j) * T + sub * kKvTok;

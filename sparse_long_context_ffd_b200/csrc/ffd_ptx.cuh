@@ -61,6 +61,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
+// Acquire load of a shared-memory int (CTA scope): later loads of this
+// thread see what the writer stored before its releasing store or fence.
+__device__ __forceinline__ int ld_acquire_cta(const volatile int *p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];"
+               : "=r"(v)
+               : "r"(smem_addr(const_cast<const int *>(p)))
+               : "memory");
+  return v;
+}
+
 // Non-blocking test of phase completion (never suspends the thread).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   uint32_t done;
