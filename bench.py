@@ -346,6 +346,23 @@ class Replica:
                 raise RuntimeError(f"device flags {flags:#x}")
 
 
+def error_vs_dense(rep, delta):
+    """The sparse step's output against the same kernel in dense mode
+    (delta = +inf) on the same inputs: max-abs, mean-abs and relative L2 over
+    all output elements (what the Top-delta selection costs in accuracy)."""
+    torch = rep.torch
+    out = rep.layers[0]["bufs"].out
+    rep.step(0, delta)
+    torch.cuda.synchronize(rep.device)
+    sparse = out.float().cpu().numpy().astype(np.float64)
+    rep.step(0, float("inf"))
+    torch.cuda.synchronize(rep.device)
+    dense = out.float().cpu().numpy().astype(np.float64)
+    d = sparse - dense
+    return {"max_abs": float(np.abs(d).max()), "mean_abs": float(np.abs(d).mean()),
+            "rel_l2": float(np.linalg.norm(d) / max(float(np.linalg.norm(dense)), 1e-30))}
+
+
 def time_graph_steps(rep, delta, steps, warmup, world, device, sampler=None, spg=None, fused=True):
     """Replay K steps from CUDA graphs; returns (total_ms, per-decode ms list)."""
     torch = rep.torch
@@ -741,6 +758,7 @@ def measure_thumb_resid(w, inp, device, args, world, l2):
     torch.cuda.synchronize(device)
     mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
     kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+    vs_dense = error_vs_dense(probe, w.delta)
     algo = algorithmic_bytes_tr(w, inp["lengths"], kept_tok, dense=False)
     valid_tok = int(np.sum(inp["lengths"])) * w.num_kv_heads
     algo_dense = algorithmic_bytes_tr(w, inp["lengths"], valid_tok, dense=True)
@@ -761,6 +779,7 @@ def measure_thumb_resid(w, inp, device, args, world, l2):
         "ms_per_step": dist_max(total / steps, world, device),
         "decode_us": dec * 1e3 if dec else None,
         "kept_blocks": kept_blocks, "kept_fraction": kept_blocks / max(1, valid_blocks),
+        "sparsity": 1.0 - kept_blocks / max(1, valid_blocks), "vs_dense": vs_dense,
         "algorithmic_bytes_per_launch": algo, "achieved_gbs": ach,
         "frac": ach / peak if ach else None,
         "traffic": ncu_traffic_per_launch(args.workload, dense=False, fmt="tr"),
@@ -798,6 +817,7 @@ def run_gpu(args):
     torch.cuda.synchronize(device)
     mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
     kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+    vs_dense = error_vs_dense(probe, w.delta)
     algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)
     valid_tok = int(np.sum(inp["lengths"])) * w.num_kv_heads
     algo_dense = algorithmic_bytes(w, inp["lengths"], valid_tok, dense=True)
@@ -869,6 +889,7 @@ def run_gpu(args):
                        "reference": args.reference,
                        "kept_blocks": kept_blocks, "valid_blocks": valid_blocks,
                        "kept_fraction": kept_blocks / max(1, valid_blocks),
+                       "sparsity": 1.0 - kept_blocks / max(1, valid_blocks),
                        "l2": f"inputs rotated over {layers} cache copies "
                              f"(>= 3x the {l2 >> 20} MiB L2 per cycle)",
                        "steps_per_graph": spg, "parallelism": f"replicas x{world}"},
@@ -878,6 +899,7 @@ def run_gpu(args):
                                    "re-quantisation + selector + computer + merge)",
                          "algorithmic_bytes_per_launch": algo, "launch_us": decode_ms * 1e3,
                          "peak_source": peak_src, "timing": timing_method},
+            "vs_dense": vs_dense,
             "two_launch_step": {"ms_per_step": two_total / max(1, min(args.steps, 400)),
                                 "decode_us": float(np.mean(two_per)) * 1e3 if two_per else None,
                                 "how": "ffd_quantize_keys(FFD_LAST_BLOCK) + ffd_decode"},
