@@ -247,13 +247,16 @@ def load_peaks():
         return 6650.0, "fallback 6.65 TB/s"
 
 
+# the sources the decode kernel and its launch are built from
+DECODE_SOURCES = ("api.cu", "decode.cu", "ffd_internal.h", "ffd_ptx.cuh", "ffd_quant.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_long_context_ffd_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -344,6 +347,35 @@ class Replica:
             flags = self.ffd.check_device_status(L["bufs"].workspace)
             if flags:
                 raise RuntimeError(f"device flags {flags:#x}")
+
+
+NOMINAL_HBM_GBS = 8000.0  # the B200 HBM3e figure the method's target is stated against
+
+
+def read_probe_gbs(device, gib=4, iters=20):
+    """Streaming-read bandwidth of this GPU, measured in the run by the
+    library's read probe (ffd_read_probe) over a buffer of `gib` GiB, far
+    above the L2: one-pass reads, the access kind the decode step makes."""
+    import torch
+    from sparse_long_context_ffd_b200 import ffd
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
+    for _ in range(3):
+        ffd.read_probe(buf, sink)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    start.record()
+    for _ in range(iters):
+        ffd.read_probe(buf, sink)
+    end.record()
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end) / iters
+    del buf
+    return buf_bytes_gbs(gib << 30, ms)
+
+
+def buf_bytes_gbs(nbytes, ms):
+    return nbytes / (ms * 1e-3) / 1e9
 
 
 def error_vs_dense(rep, delta):
@@ -853,6 +885,7 @@ def run_gpu(args):
     peak, peak_src = load_peaks()
     achieved = algo["total"] / (decode_ms * 1e-3) / 1e9
     traffic = ncu_traffic_per_launch(args.workload, dense=False)
+    probe_gbs = read_probe_gbs(device)
 
     tr = None
     if not args.no_tr:
@@ -898,7 +931,11 @@ def run_gpu(args):
                          "kernel": "ffd decode_kernel via ffd_decode_step (last-block "
                                    "re-quantisation + selector + computer + merge)",
                          "algorithmic_bytes_per_launch": algo, "launch_us": decode_ms * 1e3,
-                         "peak_source": peak_src, "timing": timing_method},
+                         "peak_source": peak_src, "timing": timing_method,
+                         "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
+                         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                         "read_probe": "ffd_read_probe over 4 GiB in this run (one-pass "
+                                       "16-byte loads, L1 no-allocate)"},
             "vs_dense": vs_dense,
             "two_launch_step": {"ms_per_step": two_total / max(1, min(args.steps, 400)),
                                 "decode_us": float(np.mean(two_per)) * 1e3 if two_per else None,

@@ -369,6 +369,16 @@ const char *ffd_status_string(ffd_status status);
 /* ABI version of this library (bumped on any incompatible change). */
 int32_t ffd_abi_version(void);
 
+/* Streaming-read bandwidth probe (not part of the method; a reference point
+ * for the decode kernel's roofline, which is a one-pass read of HBM).  Reads
+ * `bytes` of device memory at `buf` once with 16-byte loads that do not
+ * allocate in L1, on `cuda_stream`; time it with events around the call.
+ * `sink` (device, one uint32) is written only if the data fold to a fixed
+ * constant, so that no load can be elided.  buf must be 16-byte aligned and
+ * bytes a non-zero multiple of 16 (else FFD_ERR_INVALID_ARG, nothing
+ * launched).  Use a buffer well above the 126 MB L2 to measure HBM. */
+ffd_status ffd_read_probe(const void *buf, size_t bytes, uint32_t *sink, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

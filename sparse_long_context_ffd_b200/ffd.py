@@ -37,6 +37,7 @@ EXPORTED = (
     "ffd_thumb_bytes", "ffd_residual_bytes", "ffd_quantize_keys_tr", "ffd_decode_tr",
     "ffd_decode_partials_tr", "ffd_decode_append", "ffd_decode_append_tr",
     "ffd_step_graph_create", "ffd_step_graph_run", "ffd_step_graph_destroy",
+    "ffd_read_probe",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -138,6 +139,8 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_decode_no_alloc.restype = st
             lib.ffd_check_device_status.argtypes = [p, ctypes.POINTER(ctypes.c_uint32), p]
             lib.ffd_check_device_status.restype = st
+            lib.ffd_read_probe.argtypes = [p, sz, p, p]
+            lib.ffd_read_probe.restype = st
             lib.ffd_status_string.argtypes = [st]
             lib.ffd_status_string.restype = ctypes.c_char_p
             lib.ffd_abi_version.argtypes = []
@@ -349,6 +352,13 @@ def decode_no_alloc(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: f
                                               _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
                                               float(delta), _ptr(out), _ptr(mask),
                                               _stream(stream)), "ffd_decode_no_alloc")
+
+
+def read_probe(buf, sink, stream=None) -> None:
+    """ffd_read_probe: read the whole (16-byte aligned) device tensor `buf`
+    once; `sink` is a device int32/uint32 tensor of at least one element."""
+    _check(load_library().ffd_read_probe(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink),
+                                         _stream(stream)), "ffd_read_probe")
 
 
 def check_device_status(workspace, stream=None) -> int:

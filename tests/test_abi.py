@@ -231,3 +231,13 @@ def test_binding_has_no_cpu_fallback():
     t = torch.zeros(16, dtype=torch.uint8)
     with pytest.raises(ValueError):
         ffd.decode(s, t, t, t, t, t, t, 1.0, t, t, t)
+
+
+def test_read_probe_rejects_bad_arguments_on_host():
+    lib = ffd.load_library()
+    a = 1 << 20  # never dereferenced: every call below fails its host checks
+    assert lib.ffd_read_probe(None, 1024, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_read_probe(a, 1024, None, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_read_probe(a, 0, a, None) == ffd.FFD_ERR_INVALID_ARG
+    assert lib.ffd_read_probe(a, 1000, a, None) == ffd.FFD_ERR_INVALID_ARG  # not a multiple of 16
+    assert lib.ffd_read_probe(a + 8, 1024, a, None) == ffd.FFD_ERR_INVALID_ARG  # misaligned
