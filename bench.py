@@ -626,6 +626,20 @@ def _oracle_unit_worker(args):
     return time.perf_counter() - t0
 
 
+def host_cpu() -> dict:
+    """The host the oracle ran on: CPU model and logical CPU count."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
 def oracle_parallel_sample(w, inp, budget_s: float):
     """The oracle as it stands, on several host cores at once: one process per
     kv-head group of sequence 0 (independent units of the step), each over the
@@ -687,7 +701,7 @@ def run_reference(args):
         "data": "synthetic (seeded generator; stands in for RULER/LongBench inputs)",
         "config": {"workload": w.description, "name": w.name},
         "cpu_baseline": {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": desc, "single_thread_value": single_us,
+                         "sample": desc, "host": host_cpu(), "single_thread_value": single_us,
                          "single_thread_sample": desc1},
         "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -906,6 +920,7 @@ def run_gpu(args):
         us1, desc1, used = oracle_step_sample(w, inp, args.cpu_budget)
         us, cores, desc = oracle_parallel_sample(w, inp, args.cpu_budget)
         cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+               "host": host_cpu(),
                "single_thread_value": us1,
                "single_thread_sample": desc1 + f"; {used:.1f} s of CPU time"}
 
@@ -931,6 +946,7 @@ def run_gpu(args):
                          "kernel": "ffd decode_kernel via ffd_decode_step (last-block "
                                    "re-quantisation + selector + computer + merge)",
                          "algorithmic_bytes_per_launch": algo, "launch_us": decode_ms * 1e3,
+                         "launch_us_median": float(np.median(per_decode)) * 1e3,
                          "peak_source": peak_src, "timing": timing_method,
                          "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
                          "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
