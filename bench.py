@@ -872,8 +872,7 @@ def run_gpu(args):
     rep = Replica(w, inp, device, layers)
     rep.reference = REFERENCES[args.reference]
 
-    sampler = ClockSampler(device.index, os.path.join(ROOT, "gpurun_out", "clocks.csv")
-                           if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    sampler = ClockSampler(device.index, args.clocks_csv)
     sampler.start()
     time.sleep(0.8)  # let nvidia-smi start before the measured window
     total_ms, per_decode, spg = time_graph_steps(rep, w.delta, args.steps, args.warmup, world,
@@ -994,6 +993,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ffd", "reference"], default="ffd")
     ap.add_argument("--workload", choices=sorted(fw.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--delta", type=float, default=None)
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the raw nvidia-smi clock samples of the timed window here")
     ap.add_argument("--reference", choices=sorted(REFERENCES), default="running",
                     help="Top-delta reference maximum: running max in the split, or the "
                          "pseudo-max of the sink and local blocks")

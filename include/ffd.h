@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   FFD_OK = 0,
   FFD_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad shape, NaN or negative delta */
-  FFD_ERR_UNSUPPORTED = 2,  /* a valid shape this build does not implement */
+  FFD_ERR_UNSUPPORTED = 2,  /* a valid shape this library does not implement */
   FFD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than ffd_decode_workspace_bytes */
   FFD_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, tensor map) */
   FFD_ERR_DEVICE_CHECK = 5, /* ffd_check_device_status found a device-side error flag */
@@ -75,7 +75,7 @@ typedef enum {
 /* block_begin value for ffd_quantize_keys: each sequence's last block only. */
 #define FFD_LAST_BLOCK (-1)
 
-/* Largest split size (blocks) this build accepts. */
+/* Largest split size (blocks) this library accepts. */
 #define FFD_MAX_SPLIT_BLOCKS 512
 
 typedef struct {

@@ -1078,7 +1078,7 @@ size_t smem_bytes_tf(int split_blocks) {
 }
 
 // Raise the kernel's dynamic shared memory cap once per device, to the
-// largest split this build accepts, so later launches (and graph captures)
+// largest split this library accepts, so later launches (and graph captures)
 // need no attribute call.
 template <int T, int G, int F>
 cudaError_t configure_tgf() {
