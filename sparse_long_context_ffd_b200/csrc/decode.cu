@@ -994,13 +994,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       p.mask[row * p.mask_words + w] = 0u;
   }
   if (p.partials_only) return;  // context shard: the merge runs after the exchange
-  __threadfence();
+  // Split counter: the barrier, then one acquire-release add, publishes this
+  // CTA's partial and mask words; the CTA that brings the count to nsplit
+  // merges, its loads ordered after every other split's by the same add.
   named_barrier(1, kAttnThreads);
   if (threadIdx.x == 0)
-    ctrl[2] = atomicAdd(&p.counters[row], 1u) == static_cast<unsigned>(nsplit - 1) ? 1 : 0;
+    ctrl[2] = atomic_add_acq_rel_gpu(&p.counters[row], 1u) == static_cast<uint32_t>(nsplit - 1) ? 1 : 0;
   named_barrier(1, kAttnThreads);
   if (!ctrl[2]) return;
-  __threadfence();
 
   // last CTA of (b, g): log-sum-exp merge over the splits.  Warp w merges
   // heads w, w + 4 (lane: output channels 4*lane .. 4*lane + 3).  Per chunk of

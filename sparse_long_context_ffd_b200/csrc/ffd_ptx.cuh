@@ -72,6 +72,16 @@ __device__ __forceinline__ int ld_acquire_cta(const volatile int *p) {
   return v;
 }
 
+// Atomic add with acquire-release semantics at GPU scope; returns the old
+// value.  After a CTA barrier, one thread's release publishes the writes of
+// every thread of the CTA made before the barrier, and its acquire (then a
+// barrier) orders the CTA's later loads after what the other CTAs published.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Non-blocking test of phase completion (never suspends the thread).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   uint32_t done;
