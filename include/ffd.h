@@ -65,7 +65,7 @@ typedef enum {
   FFD_ERR_WORKSPACE = 3,    /* workspace missing or smaller than ffd_decode_workspace_bytes */
   FFD_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, copy, tensor map) */
   FFD_ERR_DEVICE_CHECK = 5, /* ffd_check_device_status found a device-side error flag */
-  FFD_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up */
+  FFD_ERR_TIMEOUT = 6       /* a bounded device wait gave up (ffd_check_device_status) */
 } ffd_status;
 
 /* Device-side error flags, reported by ffd_check_device_status. */
@@ -180,6 +180,13 @@ typedef struct {
   int32_t reference;
   /* 1: re-quantise each sequence's last block first, as ffd_decode_step. */
   int32_t requant_last;
+  /* Longest wait, in microseconds, of any pipeline barrier or selection-queue
+   * wait inside the kernel; a wait that runs out sets FFD_DEVICE_FLAG_TIMEOUT
+   * and the kernel finishes without a valid result (ffd_check_device_status
+   * then returns FFD_ERR_TIMEOUT).  0: the default of 2 s; negative values
+   * are rejected.  The kernel's waits for its own copies still in flight use
+   * the default in every case. */
+  int32_t wait_limit_us;
 } ffd_decode_options;
 
 /* ffd_decode / ffd_decode_step with options (NULL is rejected).  k_packed
@@ -360,7 +367,8 @@ ffd_status ffd_decode_no_alloc(const ffd_shape *shape, const void *q_bf16, const
 
 /* Synchronise the stream, read and clear the workspace's sticky device error
  * word.  *flags_out (may be NULL) receives FFD_DEVICE_FLAG_* bits.  Returns
- * FFD_ERR_DEVICE_CHECK if any flag was set, FFD_ERR_CUDA on a CUDA error. */
+ * FFD_ERR_TIMEOUT if FFD_DEVICE_FLAG_TIMEOUT was set, else
+ * FFD_ERR_DEVICE_CHECK if any other flag was, FFD_ERR_CUDA on a CUDA error. */
 ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream);
 
 /* Static description of a status code. */

@@ -14,7 +14,7 @@ namespace ffd {
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -251,7 +251,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
                          int32_t reference, bool partials_only = false, const void *k_new = nullptr,
-                         const void *v_new = nullptr) {
+                         const void *v_new = nullptr, uint64_t wait_limit_ns = kWaitLimitNs) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL)
@@ -319,6 +319,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   p.requant_last = requant ? 1 : 0;
   p.reference = reference;
   p.partials_only = partials_only ? 1 : 0;
+  p.wait_limit_ns = wait_limit_ns;
   p.k = static_cast<const uint16_t *>(kb.k);
   p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(kb.packed)) : nullptr;
   p.scales_out = requant ? static_cast<uint16_t *>(const_cast<void *>(kb.scales)) : nullptr;
@@ -346,7 +347,11 @@ KeyBuffers tr_keys(const void *k, const void *thumb, const void *resid, const vo
 }
 
 bool options_ok(const ffd_decode_options *opt) {
-  return opt != nullptr && (opt->requant_last == 0 || opt->requant_last == 1);
+  return opt != nullptr && (opt->requant_last == 0 || opt->requant_last == 1) && opt->wait_limit_us >= 0;
+}
+
+uint64_t wait_limit(const ffd_decode_options *opt) {
+  return opt->wait_limit_us > 0 ? static_cast<uint64_t>(opt->wait_limit_us) * 1000u : kWaitLimitNs;
 }
 
 }  // namespace
@@ -374,7 +379,7 @@ ffd_status ffd_decode_partials(const ffd_shape *s, const ffd_decode_options *opt
   if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
   return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_local_lengths, delta,
                        nullptr, nullptr, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
-                       opt->reference, true);
+                       opt->reference, true, nullptr, nullptr, wait_limit(opt));
 }
 
 ffd_status ffd_decode_partials_tr(const ffd_shape *s, const ffd_decode_options *opt, const void *q_bf16,
@@ -384,7 +389,7 @@ ffd_status ffd_decode_partials_tr(const ffd_shape *s, const ffd_decode_options *
   if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
   return decode_common(s, q_bf16, tr_keys(k_bf16, k_thumb, k_resid, k_scales), v_bf16, d_local_lengths,
                        delta, nullptr, nullptr, workspace, workspace_bytes, cuda_stream,
-                       opt->requant_last == 1, opt->reference, true);
+                       opt->requant_last == 1, opt->reference, true, nullptr, nullptr, wait_limit(opt));
 }
 
 ffd_status ffd_partials_region(const ffd_shape *s, size_t *offset, size_t *bytes) {
@@ -445,7 +450,7 @@ ffd_status ffd_decode_ex(const ffd_shape *s, const ffd_decode_options *opt, cons
   if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
   return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
                        mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
-                       opt->reference);
+                       opt->reference, false, nullptr, nullptr, wait_limit(opt));
 }
 
 ffd_status ffd_decode_append(const ffd_shape *s, int32_t reference, const void *q_bf16,
@@ -475,7 +480,7 @@ ffd_status ffd_decode_tr(const ffd_shape *s, const ffd_decode_options *opt, cons
   if (!options_ok(opt)) return FFD_ERR_INVALID_ARG;
   return decode_common(s, q_bf16, tr_keys(k_bf16, k_thumb, k_resid, k_scales), v_bf16, d_lengths, delta,
                        out_bf16, mask, workspace, workspace_bytes, cuda_stream, opt->requant_last == 1,
-                       opt->reference);
+                       opt->reference, false, nullptr, nullptr, wait_limit(opt));
 }
 
 ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *cuda_stream) {
@@ -491,6 +496,7 @@ ffd_status ffd_check_device_status(void *workspace, uint32_t *flags_out, void *c
       return FFD_ERR_CUDA;
   }
   if (flags_out) *flags_out = flags;
+  if (flags & FFD_DEVICE_FLAG_TIMEOUT) return FFD_ERR_TIMEOUT;
   return flags != 0 ? FFD_ERR_DEVICE_CHECK : FFD_OK;
 }
 

@@ -135,11 +135,11 @@ __device__ __forceinline__ void raise_timeout(const DecodeParams &p, volatile in
 }
 
 // Spin (bounded) until the producer has published item `it` in a stage.
-__device__ __forceinline__ bool wait_item_published(volatile int *seq, int st, int it) {
+__device__ __forceinline__ bool wait_item_published(volatile int *seq, int st, int it, uint64_t limit_ns) {
   if (seq[st] == it) return true;
   const uint64_t t0 = global_timer_ns();
   while (seq[st] != it) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
     __nanosleep(20);
   }
   return true;
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint64_t now = global_timer_ns();
         if (idle_since == 0) {
           idle_since = now;
-        } else if (now - idle_since > kWaitLimitNs) {
+        } else if (now - idle_since > p.wait_limit_ns) {
           raise_timeout(p, ctrl);
           break;
         }
@@ -640,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     for (int e = 0; e < nref + nbs; ++e) {
       const int st = e % NSA;
-      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, kWaitLimitNs)) {
+      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, p.wait_limit_ns)) {
         raise_timeout(p, ctrl);
         break;
       }
@@ -767,8 +767,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // a parity wait could then match that older phase.  The producer writes
     // `it` into seq[st] only after the previous fill was consumed, so once it
     // is visible the parity below names exactly this fill.
-    if (!wait_item_published(seq, st, it) ||
-        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / NKV) & 1u, kWaitLimitNs)) {
+    if (!wait_item_published(seq, st, it, p.wait_limit_ns) ||
+        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / NKV) & 1u, p.wait_limit_ns)) {
       raise_timeout(p, ctrl);
       break;
     }

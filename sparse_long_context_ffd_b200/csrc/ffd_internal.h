@@ -62,6 +62,9 @@ struct DecodeParams {
   // context sharding: write the split partials and bits only (no final merge;
   // out and mask unused)
   int32_t partials_only;
+  // limit of the pipeline and queue waits (the drains of the kernel's own
+  // copies always use kWaitLimitNs)
+  uint64_t wait_limit_ns;
 };
 
 // Merge of split partials gathered from num_shards context shards.

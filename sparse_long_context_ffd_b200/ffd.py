@@ -54,7 +54,8 @@ class FFDError(RuntimeError):
 
 
 class DecodeOptions(ctypes.Structure):
-    _fields_ = [("reference", ctypes.c_int32), ("requant_last", ctypes.c_int32)]
+    _fields_ = [("reference", ctypes.c_int32), ("requant_last", ctypes.c_int32),
+                ("wait_limit_us", ctypes.c_int32)]
 
 
 class Shape(ctypes.Structure):
@@ -230,10 +231,10 @@ def quantize_keys_tr(shape: Shape, k, lengths, block_begin: int, k_thumb, k_resi
 
 def decode_tr(shape: Shape, q, k, v, k_thumb, k_resid, k_scales, lengths, delta: float, out,
               mask, workspace, reference: int = FFD_REFERENCE_RUNNING_MAX,
-              requant_last: bool = False, stream=None) -> None:
+              requant_last: bool = False, stream=None, wait_limit_us: int = 0) -> None:
     """Decode step on the thumbnail + residual key format (k is read only when
     requant_last re-quantises the last block; it may be None otherwise)."""
-    opts = DecodeOptions(int(reference), 1 if requant_last else 0)
+    opts = DecodeOptions(int(reference), 1 if requant_last else 0, int(wait_limit_us))
     _check(load_library().ffd_decode_tr(ctypes.byref(shape), ctypes.byref(opts), _ptr(q), _ptr(k),
                                          _ptr(v), _ptr(k_thumb), _ptr(k_resid), _ptr(k_scales),
                                          _ptr(lengths), float(delta), _ptr(out), _ptr(mask),
@@ -302,9 +303,10 @@ def decode_step(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float
 
 def decode_ex(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: float, out, mask,
               workspace, reference: int = FFD_REFERENCE_RUNNING_MAX, requant_last: bool = False,
-              stream=None) -> None:
-    """ffd_decode / ffd_decode_step with the reference-maximum mode."""
-    opts = DecodeOptions(int(reference), 1 if requant_last else 0)
+              stream=None, wait_limit_us: int = 0) -> None:
+    """ffd_decode / ffd_decode_step with the reference-maximum mode and the
+    kernel's wait limit (0: the default 2 s; see ffd_decode_options)."""
+    opts = DecodeOptions(int(reference), 1 if requant_last else 0, int(wait_limit_us))
     _check(load_library().ffd_decode_ex(ctypes.byref(shape), ctypes.byref(opts), _ptr(q), _ptr(k),
                                          _ptr(v), _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
                                          float(delta), _ptr(out), _ptr(mask), _ptr(workspace),
@@ -366,7 +368,7 @@ def check_device_status(workspace, stream=None) -> int:
     flags = ctypes.c_uint32(0)
     st = load_library().ffd_check_device_status(_ptr(workspace), ctypes.byref(flags),
                                                 _stream(stream))
-    if st not in (FFD_OK, FFD_ERR_DEVICE_CHECK):
+    if st not in (FFD_OK, FFD_ERR_DEVICE_CHECK, FFD_ERR_TIMEOUT):
         raise FFDError(st, "ffd_check_device_status")
     return int(flags.value)
 

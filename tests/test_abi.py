@@ -41,7 +41,7 @@ def test_build_targets_sm100a():
 
 
 def test_abi_version_and_status_strings():
-    assert ffd.abi_version() == 1
+    assert ffd.abi_version() == 2
     assert ffd.status_string(ffd.FFD_OK) == "ok"
     for code in range(1, 7):
         assert ffd.status_string(code) not in ("ok", "unknown status")
@@ -120,7 +120,8 @@ def test_bad_arguments_rejected_on_host():
                                None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_decode_step(ctypes.byref(s), a, a, a, a, a, a, -1.0, a, a, a, ws,
                                None) == ffd.FFD_ERR_INVALID_ARG
-    for bad in (ffd.DecodeOptions(2, 0), ffd.DecodeOptions(-1, 0), ffd.DecodeOptions(0, 2)):
+    for bad in (ffd.DecodeOptions(2, 0), ffd.DecodeOptions(-1, 0), ffd.DecodeOptions(0, 2),
+                ffd.DecodeOptions(0, 0, -1)):
         assert lib.ffd_decode_ex(ctypes.byref(s), ctypes.byref(bad), a, a, a, a, a, a, 1.0, a, a,
                                  a, ws, None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_decode_ex(ctypes.byref(s), None, a, a, a, a, a, a, 1.0, a, a, a, ws,
