@@ -16,6 +16,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libffd_b200.so")
+# the same sources with FFD_DEBUG: every global index the decode kernel
+# computes is bounds-checked and flagged (FFD_DEVICE_FLAG_BOUNDS); for tests
+DEBUG_LIB = os.path.join(PKG, "libffd_b200_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
@@ -31,10 +34,11 @@ def _inputs():
         glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(path: str = None) -> bool:
+    path = path or LIB
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
@@ -45,20 +49,22 @@ def nvcc() -> str:
     return path
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not is_stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    target = DEBUG_LIB if debug else LIB
+    if not force and not is_stale(target):
+        return target
+    tmp = target + f".tmp{os.getpid()}"
+    flags = [*extra, "-DFFD_DEBUG"] if debug else list(extra)
+    cmd = [nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *flags, "-I", INCLUDE, "-I", CSRC,
            "-cudart", "static", "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else ())
-    print(LIB)
+    debug = "--debug" in sys.argv
+    print(build(force="--force" in sys.argv, verbose=True,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else (), debug=debug))

@@ -42,6 +42,17 @@ namespace ffd {
 namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+// Debug build (FFD_DEBUG): every global index the kernel computes is checked
+// against the extent the shape implies; a violation sets kFlagBounds in the
+// sticky word and the access is skipped (a skipped copy leaves its barrier
+// short, so the waits end at their limit).  Without FFD_DEBUG the checks
+// compile away.
+#ifdef FFD_DEBUG
+#define FFD_IN_BOUNDS(params, cond) ((cond) || (atomicOr((params).err, kFlagBounds), false))
+#else
+#define FFD_IN_BOUNDS(params, cond) true
+#endif
 constexpr float kRsqrtD = 0.08838834764831845f;     // nearest float to 1/sqrt(128)
 constexpr float kFltMax = 3.4028234663852886e38f;
 constexpr float kScaleLog2 = 0.12751743074195287f;  // log2(e) / sqrt(128)
@@ -432,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // Empty or invalid sequence: split 0 writes zero rows and an empty mask.
     if (split == 0) {
       if (bad && threadIdx.x == 0 && g == 0) atomicOr(p.err, kFlagBadLength);
-      if (!p.partials_only) {  // (a context shard leaves the rows to the merge)
+      if (!p.partials_only &&
+          FFD_IN_BOUNDS(p, row < static_cast<size_t>(p.batch) * p.num_kv_heads)) {  // (a shard leaves them to the merge)
         for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) out_rows[i] = 0;
         for (int w = threadIdx.x; w < p.mask_words; w += blockDim.x) p.mask[row * p.mask_words + w] = 0u;
       }
@@ -485,6 +497,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint8_t *src_p = p.packed + row * p.capacity * SG::kRowBytes;
     const uint16_t *src_s = p.scales + row * static_cast<size_t>(p.capacity / T) * kHeadDim;
     const int row_tok0 = static_cast<int>(row * p.capacity);
+    const bool row_ok = row < static_cast<size_t>(p.batch) * p.num_kv_heads;
+    (void)row_ok;
     const int scan_total = dense ? 0 : nref + nbs;
     int sc_next = 0;                // scan tiles issued
     int it_next = 0;                // attention stages issued (items + end markers)
@@ -518,10 +532,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
         uint8_t *dst = scan_ring + st * SG::kStageBytes;
         mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
-        bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * SG::kRowBytes, T * SG::kRowBytes,
-                 &full_a[st]);
-        bulk_g2s(dst + T * SG::kRowBytes, src_s + static_cast<size_t>(jb) * kHeadDim,
-                 kScaleRowBytes, &full_a[st]);
+        if (FFD_IN_BOUNDS(p, jb >= 0 && (jb + 1) * T <= p.capacity && row_ok)) {
+          bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * SG::kRowBytes, T * SG::kRowBytes,
+                   &full_a[st]);
+          bulk_g2s(dst + T * SG::kRowBytes, src_s + static_cast<size_t>(jb) * kHeadDim,
+                   kScaleRowBytes, &full_a[st]);
+        }
         ++sc_next;
         progress = true;
       }
@@ -547,16 +563,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         seq[st] = it_next;
         mbar_arrive_expect_tx(&full_b[st], KG::kTx);
         const int y = row_tok0 + tok;
-        if constexpr (kTR) {
-          tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);  // residual rows
-          bulk_g2s(dst + KG::kThumbOffset, src_p + static_cast<size_t>(tok) * kThumbRowBytes,
-                   kKvTok * kThumbRowBytes, &full_b[st]);
-          bulk_g2s(dst + KG::kScaleOffset, src_s + static_cast<size_t>(tok / T) * kHeadDim,
-                   kScaleRowBytes, &full_b[st]);
-        } else {
-          tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);  // K: both halves
+        if (FFD_IN_BOUNDS(p, tok >= 0 && tok + kKvTok <= p.capacity && row_ok)) {
+          if constexpr (kTR) {
+            tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);  // residual rows
+            bulk_g2s(dst + KG::kThumbOffset, src_p + static_cast<size_t>(tok) * kThumbRowBytes,
+                     kKvTok * kThumbRowBytes, &full_b[st]);
+            bulk_g2s(dst + KG::kScaleOffset, src_s + static_cast<size_t>(tok / T) * kHeadDim,
+                     kScaleRowBytes, &full_b[st]);
+          } else {
+            tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);  // K: both halves
+          }
+          tma_load_3d(dst + KG::kVOffset, &tmap_v, 0, y, 0, &full_b[st]);  // V: both halves
         }
-        tma_load_3d(dst + KG::kVOffset, &tmap_v, 0, y, 0, &full_b[st]);  // V: both halves
         ++it_next;
         ++sub;
         progress = true;
@@ -695,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // releases the producer
     const int jl = nb - 1;
     const size_t tok0 = row * static_cast<size_t>(p.capacity) + static_cast<size_t>(jl) * T;
-    if (new_k_row != nullptr && threadIdx.x < 32) {
+    if (new_k_row != nullptr && threadIdx.x < 32 && FFD_IN_BOUNDS(p, len >= 1 && len <= p.capacity)) {
       const size_t at = (row * static_cast<size_t>(p.capacity) + static_cast<size_t>(len - 1)) * kHeadDim;
       const int c = threadIdx.x & 15;
       if (threadIdx.x < 16)
@@ -705,17 +723,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     float *red = reinterpret_cast<float *>(smem + SL::kRequant);
     uint16_t *scale_row = p.scales_out + (row * static_cast<size_t>(p.capacity / T) + jl) * kHeadDim;
-    if constexpr (kTR)
-      quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
-                                         p.packed_out + tok0 * kThumbRowBytes,
-                                         p.resid_out + tok0 * kResidRowBytes, scale_row, red,
-                                         red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
-                                         new_k_row);
-    else
-      quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
-                                      p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
-                                      red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
-                                      new_k_row);
+    // (the condition is the same in every attention thread: the quantiser's
+    // named barriers stay matched)
+    if (FFD_IN_BOUNDS(p, jl >= 0 && (jl + 1) * T <= p.capacity &&
+                             row < static_cast<size_t>(p.batch) * p.num_kv_heads)) {
+      if constexpr (kTR)
+        quantize_block_tr<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                           p.packed_out + tok0 * kThumbRowBytes,
+                                           p.resid_out + tok0 * kResidRowBytes, scale_row, red,
+                                           red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
+                                           new_k_row);
+      else
+        quantize_block<T, kAttnThreads>(p.k + tok0 * kHeadDim, min(T, len - jl * T),
+                                        p.packed_out + tok0 * kPackedRowBytes, scale_row, red,
+                                        red + kAttnWarps * kHeadDim, static_cast<int>(threadIdx.x), 2,
+                                        new_k_row);
+    }
     fence_proxy_async_global();
     __threadfence_block();
     named_barrier(2, kAttnThreads);
@@ -955,6 +978,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   named_barrier(1, kAttnThreads);
   const size_t unit = row * p.nsplit_max + split;
   float *part = p.partials + unit * G * kPartialStride;
+  const bool unit_ok =
+      FFD_IN_BOUNDS(p, unit < static_cast<size_t>(p.batch) * p.num_kv_heads * p.nsplit_max && split < p.nsplit_max);
   for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAttnThreads) {
     const int h = idx >> 7, c = idx & 127;
     float M = -INFINITY;
@@ -970,10 +995,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         A += wacc[(w * 8 + h) * kHeadDim + c] * f;
       }
     }
-    part[h * kPartialStride + c] = A;
-    if (c == 0) {
-      part[h * kPartialStride + 128] = M;
-      part[h * kPartialStride + 129] = L;
+    if (unit_ok) {
+      part[h * kPartialStride + c] = A;
+      if (c == 0) {
+        part[h * kPartialStride + 128] = M;
+        part[h * kPartialStride + 129] = L;
+      }
     }
   }
   if (static_cast<int>(threadIdx.x) < p.split_words) {
@@ -982,7 +1009,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int lo = 32 * threadIdx.x;
       bits = lo >= nbs ? 0u : (nbs - lo >= 32 ? kFull : ((1u << (nbs - lo)) - 1u));
     }
-    p.split_bits[unit * p.split_words + threadIdx.x] = bits;
+    if (unit_ok) p.split_bits[unit * p.split_words + threadIdx.x] = bits;
     // splits of a multiple of 32 blocks own whole mask words: write them here
     // rather than gather them in the final merge
     if (!p.partials_only && (p.split_blocks & 31) == 0 && (j0 >> 5) + static_cast<int>(threadIdx.x) < p.mask_words)
@@ -1057,7 +1084,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const uint32_t lo = pack_bf16x2(O.x * inv, O.y * inv), hi = pack_bf16x2(O.z * inv, O.w * inv);
-    *reinterpret_cast<uint2 *>(out_rows + h * kHeadDim + 4 * lane) = make_uint2(lo, hi);
+    if (FFD_IN_BOUNDS(p, row < static_cast<size_t>(p.batch) * p.num_kv_heads))
+      *reinterpret_cast<uint2 *>(out_rows + h * kHeadDim + 4 * lane) = make_uint2(lo, hi);
   }
   // mask row (splits not a multiple of 32 blocks): each word gathers 32
   // consecutive blocks' bits from the split bit rows
@@ -1139,6 +1167,15 @@ cudaError_t launch_f(const DecodeParams &p, const CUtensorMap &tk, const CUtenso
 
 }  // namespace
 
+#ifdef FFD_DEBUG
+namespace {
+// Evaluates a failing bounds check, as a kernel index bug would.
+__global__ void bounds_selftest_kernel(DecodeParams p) {
+  if (threadIdx.x == 0 && FFD_IN_BOUNDS(p, p.batch < 0)) p.err[1] = 0u;
+}
+}  // namespace
+#endif
+
 size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format) {
   (void)group;
   if (format == kFormatThumbResid)
@@ -1167,3 +1204,16 @@ cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, cons
 }
 
 }  // namespace ffd
+
+#ifdef FFD_DEBUG
+// Debug library only (not in the public header): sets FFD_DEVICE_FLAG_BOUNDS
+// in the workspace's sticky word through the same check the kernel uses.
+extern "C" ffd_status ffd_debug_bounds_selftest(void *workspace, void *cuda_stream) {
+  if (workspace == nullptr) return FFD_ERR_INVALID_ARG;
+  ffd::DecodeParams p{};
+  p.err = static_cast<uint32_t *>(workspace);
+  p.batch = 1;
+  ffd::bounds_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FFD_OK : FFD_ERR_CUDA;
+}
+#endif

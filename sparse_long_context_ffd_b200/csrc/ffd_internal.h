@@ -29,6 +29,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded mbarrier waits (2 s
 
 constexpr uint32_t kFlagBadLength = 0x1u;
 constexpr uint32_t kFlagTimeout = 0x2u;
+constexpr uint32_t kFlagBounds = 0x4u;  // debug build only: an index left its extent
 
 struct DecodeParams {
   const uint16_t *q;       // bf16 [B][Hq][D]

@@ -25,6 +25,7 @@ FFD_ERR_TIMEOUT = 6
 
 FFD_DEVICE_FLAG_BAD_LENGTH = 0x1
 FFD_DEVICE_FLAG_TIMEOUT = 0x2
+FFD_DEVICE_FLAG_BOUNDS = 0x4  # debug build only (FFD_DEBUG_LIBRARY=1)
 FFD_LAST_BLOCK = -1
 FFD_MAX_SPLIT_BLOCKS = 512
 
@@ -77,18 +78,25 @@ _lock = threading.Lock()
 _lib = None
 
 
+def _debug_requested() -> bool:
+    return os.environ.get("FFD_DEBUG_LIBRARY", "") in ("1", "true", "yes")
+
+
 def library_path() -> str:
-    return _build.LIB
+    """The library this process loads: libffd_b200.so, or with the environment
+    variable FFD_DEBUG_LIBRARY=1 the bounds-checking debug build."""
+    return _build.DEBUG_LIB if _debug_requested() else _build.LIB
 
 
 def load_library() -> ctypes.CDLL:
-    """Load libffd_b200.so, building it with nvcc first if it is missing or stale."""
+    """Load the library, building it with nvcc first if it is missing or stale."""
     global _lib
     with _lock:
         if _lib is None:
-            if _build.is_stale():
-                _build.build()
-            lib = ctypes.CDLL(_build.LIB)
+            path = library_path()
+            if _build.is_stale(path):
+                _build.build(debug=_debug_requested())
+            lib = ctypes.CDLL(path)
             sp = ctypes.POINTER(Shape)
             p, sz, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
             for name in ("ffd_packed_bytes", "ffd_scale_bytes", "ffd_mask_words",

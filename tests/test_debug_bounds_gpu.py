@@ -1,0 +1,23 @@
+"""The bounds-checking debug build (FFD_DEBUG) stands in for a memory
+sanitizer: every global index the decode kernel computes is checked against
+the extent the shape implies, and a violation sets FFD_DEVICE_FLAG_BOUNDS
+instead of trapping.  The small parity cases of both key formats, the pseudo
+maximum and the fused append run on it with no flag raised and the oracle's
+results (debug_bounds_run.py, in its own process: one library per process)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def test_debug_build_raises_no_bounds_flag_on_the_parity_cases():
+    env = dict(os.environ, FFD_DEBUG_LIBRARY="1")
+    r = subprocess.run([sys.executable, os.path.join(HERE, "debug_bounds_run.py")], env=env,
+                       capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    assert "no flags" in r.stdout
