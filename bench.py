@@ -626,6 +626,22 @@ def _oracle_unit_worker(args):
     return time.perf_counter() - t0
 
 
+def oracle_vs_gpu(w, inp, gpu_out, gpu_mask, pseudo_max=False) -> dict:
+    """The oracle on the whole first kv-head group of sequence 0 (all its
+    tokens) against the GPU's output rows and mask row of the same step."""
+    import oracle
+    T, S, G = w.block_size, w.split_blocks, w.group
+    ln = np.ascontiguousarray(inp["lengths"][:1])
+    k1, v1 = inp["k"][:1, :1], inp["v"][:1, :1]
+    p1, s1 = oracle.quantize_keys(k1, ln, T)
+    out, mask, _ = oracle.decode(inp["q"][:1, :G], k1, v1, p1, s1, ln, T, S, w.delta,
+                                 pseudo_max=pseudo_max)
+    d = np.abs(out[0] - gpu_out)
+    return {"heads": f"query heads 0..{G - 1} of sequence 0 (kv-head 0), all {int(ln[0])} tokens",
+            "mask_equal": bool(np.array_equal(mask[0, 0], gpu_mask)),
+            "max_abs": float(d.max()), "mean_abs": float(d.mean())}
+
+
 def host_cpu() -> dict:
     """The host the oracle ran on: CPU model and logical CPU count."""
     model = "unknown"
@@ -863,6 +879,8 @@ def run_gpu(args):
     torch.cuda.synchronize(device)
     mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
     kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+    probe_out = probe.layers[0]["bufs"].out[0, :w.group].float().cpu().numpy().astype(np.float64)
+    probe_mask = mask[0, 0].copy()
     vs_dense = error_vs_dense(probe, w.delta)
     algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)
     valid_tok = int(np.sum(inp["lengths"])) * w.num_kv_heads
@@ -875,8 +893,10 @@ def run_gpu(args):
     sampler = ClockSampler(device.index, args.clocks_csv)
     sampler.start()
     time.sleep(0.8)  # let nvidia-smi start before the measured window
+    torch.cuda.nvtx.range_push("ffd timed decode steps")
     total_ms, per_decode, spg = time_graph_steps(rep, w.delta, args.steps, args.warmup, world,
                                                  device, sampler)
+    torch.cuda.nvtx.range_pop()
     timing_method = "graph-captured timing events around each decode launch"
     if not per_decode:
         per_decode = time_gated_decodes(rep, w.delta, min(args.steps, 64), device)
@@ -918,8 +938,10 @@ def run_gpu(args):
         oracle.build()
         us1, desc1, used = oracle_step_sample(w, inp, args.cpu_budget)
         us, cores, desc = oracle_parallel_sample(w, inp, args.cpu_budget)
+        vs_gpu = oracle_vs_gpu(w, inp, probe_out, probe_mask,
+                               pseudo_max=args.reference == "sink_local")
         cpu = {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
-               "host": host_cpu(),
+               "host": host_cpu(), "vs_gpu": vs_gpu,
                "single_thread_value": us1,
                "single_thread_sample": desc1 + f"; {used:.1f} s of CPU time"}
 
@@ -946,6 +968,8 @@ def run_gpu(args):
                                    "re-quantisation + selector + computer + merge)",
                          "algorithmic_bytes_per_launch": algo, "launch_us": decode_ms * 1e3,
                          "launch_us_median": float(np.median(per_decode)) * 1e3,
+                         "launch_us_p10": float(np.percentile(per_decode, 10)) * 1e3,
+                         "launch_us_p90": float(np.percentile(per_decode, 90)) * 1e3,
                          "peak_source": peak_src, "timing": timing_method,
                          "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
                          "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
