@@ -756,8 +756,12 @@ def run_shard_measure(args):
     from sparse_long_context_ffd_b200 import ffd, sharded
     device = torch.device("cuda", torch.cuda.current_device())
     w = fw.WORKLOADS[args.workload]
+    if args.dense:
+        args.delta = float("inf")
     if args.delta is not None:
         w = fw.scaled_workload(w, delta=args.delta)
+    if args.seed is not None:
+        w = fw.scaled_workload(w, seed=args.seed)
     W = args.shards
     sharded.check_shard_capacity(w.capacity, w.block_size, w.split_blocks)
     inp = fw.make_inputs(w)
@@ -862,8 +866,12 @@ def run_gpu(args):
     device = torch.device("cuda", local_rank if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(device)
     w = fw.WORKLOADS[args.workload]
+    if args.dense:
+        args.delta = float("inf")
     if args.delta is not None:
         w = fw.scaled_workload(w, delta=args.delta)
+    if args.seed is not None:
+        w = fw.scaled_workload(w, seed=args.seed)
     # each rank serves its own request: a different seed per replica
     w_rank = fw.scaled_workload(w, seed=w.seed + 1000 * rank) if rank else w
     inp = fw.make_inputs(w_rank)
@@ -1017,6 +1025,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ffd", "reference"], default="ffd")
     ap.add_argument("--workload", choices=sorted(fw.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--delta", type=float, default=None)
+    ap.add_argument("--dense", action="store_true", help="delta = +inf (flash-decoding over all blocks)")
+    ap.add_argument("--seed", type=int, default=None, help="input seed (default: the workload's)")
     ap.add_argument("--clocks-csv", default=None,
                     help="also write the raw nvidia-smi clock samples of the timed window here")
     ap.add_argument("--reference", choices=sorted(REFERENCES), default="running",

@@ -71,8 +71,8 @@ typedef enum {
 /* Device-side error flags, reported by ffd_check_device_status. */
 #define FFD_DEVICE_FLAG_BAD_LENGTH 0x1u /* some lengths[b] outside [0, cap] */
 #define FFD_DEVICE_FLAG_TIMEOUT 0x2u    /* a bounded barrier wait expired */
-/* Debug library only (built with FFD_DEBUG): a computed global index left the
- * extent the shape implies; that access was skipped. */
+/* Debug library only (libffd_b200_debug.so, built with FFD_DEBUG): a computed
+ * global index left the extent the shape implies; that access was skipped. */
 #define FFD_DEVICE_FLAG_BOUNDS 0x4u
 
 /* block_begin value for ffd_quantize_keys: each sequence's last block only. */

@@ -18,6 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libffd_b200.so")
 # the same sources with FFD_DEBUG: every global index the decode kernel
 # computes is bounds-checked and flagged (FFD_DEVICE_FLAG_BOUNDS); for tests
+# (ffd.use_debug_library())
 DEBUG_LIB = os.path.join(PKG, "libffd_b200_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

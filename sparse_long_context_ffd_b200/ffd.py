@@ -9,7 +9,6 @@ from __future__ import annotations
 
 import ctypes
 import math
-import os
 import threading
 from typing import Optional
 
@@ -25,7 +24,7 @@ FFD_ERR_TIMEOUT = 6
 
 FFD_DEVICE_FLAG_BAD_LENGTH = 0x1
 FFD_DEVICE_FLAG_TIMEOUT = 0x2
-FFD_DEVICE_FLAG_BOUNDS = 0x4  # debug build only (FFD_DEBUG_LIBRARY=1)
+FFD_DEVICE_FLAG_BOUNDS = 0x4  # debug build only (use_debug_library())
 FFD_LAST_BLOCK = -1
 FFD_MAX_SPLIT_BLOCKS = 512
 
@@ -78,13 +77,27 @@ _lock = threading.Lock()
 _lib = None
 
 
+_use_debug = False
+
+
+def use_debug_library() -> None:
+    """Load the bounds-checking debug build (libffd_b200_debug.so: FFD_DEBUG,
+    FFD_DEVICE_FLAG_BOUNDS) instead of the product library.  For tests; call
+    it before the process's first library call."""
+    global _use_debug
+    with _lock:
+        if _lib is not None and not _use_debug:
+            raise RuntimeError("the product library is already loaded in this process")
+        _use_debug = True
+
+
 def _debug_requested() -> bool:
-    return os.environ.get("FFD_DEBUG_LIBRARY", "") in ("1", "true", "yes")
+    return _use_debug
 
 
 def library_path() -> str:
-    """The library this process loads: libffd_b200.so, or with the environment
-    variable FFD_DEBUG_LIBRARY=1 the bounds-checking debug build."""
+    """The library this process loads: libffd_b200.so, or after
+    use_debug_library() the bounds-checking debug build."""
     return _build.DEBUG_LIB if _debug_requested() else _build.LIB
 
 

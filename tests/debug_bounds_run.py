@@ -1,4 +1,4 @@
-"""Run in a process with FFD_DEBUG_LIBRARY=1 (see test_debug_bounds_gpu.py).
+"""Run in a process of its own (see test_debug_bounds_gpu.py).
 
 Loads the bounds-checking debug build of the library and runs the small
 parity cases on both key formats, the fused append and the pseudo-max
@@ -30,7 +30,7 @@ def flags_clear(ws, what):
 
 
 def main():
-    assert os.environ.get("FFD_DEBUG_LIBRARY") == "1"
+    ffd.use_debug_library()
     assert ffd.library_path().endswith("libffd_b200_debug.so")
     lib = ffd.load_library()
     # the flag path itself: a failing check reports FFD_DEVICE_FLAG_BOUNDS
