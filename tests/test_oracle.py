@@ -650,3 +650,36 @@ def test_decode_pseudo_max_attends_over_its_mask():
         ref = _library_attention(inp["q"], inp["k"], inp["v"], inp["lengths"],
                                  _token_keep(mask, w.block_size, w.capacity))
         np.testing.assert_allclose(out, ref, atol=1e-10)
+
+
+def test_sparsity_adapts_to_attention_sharpness():
+    # Methodology 2, Adaptivity (gist.science explainer): when attention is
+    # concentrated, fewer blocks fall within delta of the peak.  Same queries,
+    # same delta: flat keys keep (nearly) every block; keys whose first block
+    # of every split dominates keep little more than those blocks.
+    T, S, G, nblk = 64, 8, 4, 64
+    cap = T * nblk
+    rng = np.random.default_rng(7)
+    q0 = rng.standard_normal(128).astype(np.float32)
+    q = np.tile(q0, (1, G, 1))                       # [1, G, 128]: one direction for the group
+    flat = (0.1 * rng.standard_normal((1, 1, cap, 128))).astype(np.float32)
+    sharp = flat.copy()
+    bump = 5.0 * np.sqrt(128.0) * q0 / np.dot(q0, q0)  # raises q.k / sqrt(D) by 5 (delta is 1)
+    for j in range(0, nblk, S):                      # the first block of every split
+        sharp[0, 0, j * T:(j + 1) * T] += bump
+    v = rng.standard_normal((1, 1, cap, 128)).astype(np.float32)
+    lengths = np.array([cap], np.int32)
+    qb, vb = fw.f32_to_bf16_bits(q), fw.f32_to_bf16_bits(v)
+    kept = {}
+    for name, k in (("flat", flat), ("sharp", sharp)):
+        kb = fw.f32_to_bf16_bits(k)
+        p, s = oracle.quantize_keys(kb, lengths, T)
+        _, mask, _ = oracle.decode(qb, kb, vb, p, s, lengths, T, S, 1.0)
+        kept[name] = oracle.mask_to_blocks(mask[0, 0], nblk)
+        th, re, sc = oracle.quantize_keys_tr(kb, lengths, T)
+        _, mask_tr, _ = oracle.decode_tr(qb, vb, th, re, sc, lengths, T, S, 1.0)
+        kept[name + "_tr"] = oracle.mask_to_blocks(mask_tr[0, 0], nblk)
+    for fmt in ("", "_tr"):
+        assert kept["flat" + fmt].sum() >= 0.9 * nblk
+        assert kept["sharp" + fmt].sum() <= nblk // S + 2
+        assert all(kept["sharp" + fmt][j] for j in range(0, nblk, S))  # the dominant blocks stay
