@@ -1017,6 +1017,59 @@ def run_gpu(args):
     return 0
 
 
+CONTEXT_SWEEP = (16384, 32768, 65536, 131072, 262144)
+
+
+def run_context_sweep(args):
+    """Decode time against context length: the long-context workload (B1, Hq32,
+    Hkv8, T64, S64, its delta, drift and needles) at each length of
+    CONTEXT_SWEEP, the fused step in sparse and in dense mode, one JSON line
+    with a row per length."""
+    import torch
+    device = torch.device("cuda", torch.cuda.current_device())
+    base = fw.WORKLOADS["long128k"]
+    l2 = getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 126 * 2**20)
+    peak, peak_src = load_peaks()
+    rows = []
+    for n in CONTEXT_SWEEP:
+        w = fw.scaled_workload(base, capacity=n, context=n)
+        inp = fw.make_inputs(w)
+        probe = Replica(w, inp, device, 1)
+        probe.step(0, w.delta)
+        torch.cuda.synchronize(device)
+        mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
+        kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+        algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)["total"]
+        algo_dense = algorithmic_bytes(w, inp["lengths"], int(np.sum(inp["lengths"])) * w.num_kv_heads,
+                                       dense=True)["total"]
+        del probe
+        layers = max(1, min(64, math.ceil(3 * l2 / min(algo, algo_dense))))
+        rep = Replica(w, inp, device, layers)
+        steps = min(args.steps, 400)
+        _, per, _ = time_graph_steps(rep, w.delta, steps, args.warmup, 1, device)
+        _, per_d, _ = time_graph_steps(rep, float("inf"), steps, args.warmup, 1, device)
+        rep.check_flags()
+        sp, de = float(np.mean(per)) * 1e3, float(np.mean(per_d)) * 1e3
+        rows.append({"context": n, "sparse_us": sp, "dense_us": de,
+                     "kept_fraction": kept_blocks / max(1, valid_blocks),
+                     "sparse_frac": algo / (sp * 1e-6) / 1e9 / peak,
+                     "dense_frac": algo_dense / (de * 1e-6) / 1e9 / peak})
+        del rep, inp
+        torch.cuda.empty_cache()
+    ctx = np.array([r["context"] for r in rows], np.float64)
+    fit = {m: [float(c) for c in np.polyfit(ctx / 1024.0, [r[m + "_us"] for r in rows], 1)]
+           for m in ("sparse", "dense")}
+    line = {"mode": "context-sweep", "metric": "us per decode launch vs context length",
+            "unit": "us",
+            "workload": "long-context shape (B1 Hq32 Hkv8 D128 T64 S64 delta 3, drift 0.05/token, "
+                        "16 needles) at each context length",
+            "peak_gbs": peak, "peak_source": peak_src,
+            "rows": rows,
+            "linear_fit_us_per_1k_tokens_and_intercept": fit}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1039,6 +1092,8 @@ def main(argv=None):
                     help="skip the thumbnail + residual format measurement")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--reference-budget", type=float, default=150.0)
+    ap.add_argument("--context-sweep", action="store_true",
+                    help="the long-context workload at 16K..256K tokens, sparse and dense (one line)")
     ap.add_argument("--shards", type=int, default=0,
                     help="time one rank's share of a context-sharded step over this many shards")
     ap.add_argument("--profile-steps", type=int, default=0,
@@ -1054,6 +1109,8 @@ def main(argv=None):
         return run_profile(args)
     if args.shards:
         return run_shard_measure(args)
+    if args.context_sweep:
+        return run_context_sweep(args)
     return run_gpu(args)
 
 
