@@ -6,6 +6,7 @@ import math
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -242,3 +243,17 @@ def test_read_probe_rejects_bad_arguments_on_host():
     assert lib.ffd_read_probe(a, 0, a, None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_read_probe(a, 1000, a, None) == ffd.FFD_ERR_INVALID_ARG  # not a multiple of 16
     assert lib.ffd_read_probe(a + 8, 1024, a, None) == ffd.FFD_ERR_INVALID_ARG  # misaligned
+
+
+def test_debug_library_switch():
+    # a fresh process may switch to the bounds-checking build before its first call;
+    # a process that already loaded the product library may not
+    code = ("from sparse_long_context_ffd_b200 import ffd; ffd.use_debug_library(); "
+            "print(ffd.library_path())")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT,
+                         check=True).stdout.strip()
+    assert out.endswith("libffd_b200_debug.so")
+    ffd.load_library()
+    with pytest.raises(RuntimeError):
+        ffd.use_debug_library()
+    assert ffd.library_path().endswith("libffd_b200.so")
