@@ -157,7 +157,8 @@ ffd_status ffd_decode(const ffd_shape *shape, const void *q_bf16, const void *k_
  * block (exactly ffd_quantize_keys with FFD_LAST_BLOCK: the caller has just
  * appended the current token's K/V at position lengths[b] - 1), then run
  * ffd_decode.  The CTA that owns a sequence's last split does the
- * re-quantisation before its scan, so no other work waits for it.
+ * re-quantisation while its scan streams the split's other blocks; only its
+ * own copies of that block wait for it, and no other CTA waits at all.
  * k_packed and k_scales are read and (for the last block) written; they are
  * required even when delta == +INFINITY.  Results are bit-identical to the
  * two calls in sequence. */
