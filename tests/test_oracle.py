@@ -351,6 +351,42 @@ def test_block_scores_within_quantisation_bound():
             assert (sc[b, h, -(-n // T):] == -np.inf).all()
 
 
+def _permute_tokens_in_blocks(x, lengths, T, rng):
+    """Shuffle the valid tokens of every block (axis 2) among themselves."""
+    y = x.copy()
+    for b in range(x.shape[0]):
+        n = int(lengths[b])
+        for j0 in range(0, n, T):
+            idx = np.arange(j0, min(j0 + T, n))
+            y[b, :, idx] = x[b, :, rng.permutation(idx)]
+    return y
+
+
+def test_scores_equivariant_under_channel_and_token_permutations():
+    # The fold is elementwise over channels with a permutation-invariant max,
+    # the integer dot products are exact and the block score is a max over the
+    # block's tokens: permuting q's and K's channels together, or the tokens
+    # inside a block, must leave every score bit-identical and permute the
+    # int4 copy and its scales with them.  (A channel paired with another
+    # channel's scale, or a token counted in the wrong block, breaks it.)
+    w, inp = _rand_case(19, B=2, G=4, Hkv=2, cap=512, lo=70, hi=512)
+    T = w.block_size
+    q, k, lengths = inp["q"], inp["k"], inp["lengths"]
+    packed, scales = oracle.quantize_keys(k, lengths, T)
+    sc = oracle.block_scores(q, packed, scales, lengths, T)
+    rng = np.random.default_rng(190)
+    perm = rng.permutation(D)
+    packed_c, scales_c = oracle.quantize_keys(np.ascontiguousarray(k[..., perm]), lengths, T)
+    assert np.array_equal(scales_c, scales[..., perm])
+    assert np.array_equal(_unpack_codes(packed_c), _unpack_codes(packed)[..., perm])
+    sc_c = oracle.block_scores(np.ascontiguousarray(q[..., perm]), packed_c, scales_c, lengths, T)
+    assert np.array_equal(sc_c, sc)
+    k_t = _permute_tokens_in_blocks(k, lengths, T, rng)
+    packed_t, scales_t = oracle.quantize_keys(k_t, lengths, T)
+    assert np.array_equal(scales_t, scales)
+    assert np.array_equal(oracle.block_scores(q, packed_t, scales_t, lengths, T), sc)
+
+
 # ---------------------------------------------------------------- selection --
 
 def _read_golden():

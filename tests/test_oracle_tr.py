@@ -254,6 +254,41 @@ def _sdpa(q, k64, v, lengths, G, token_keep=None):
     return out
 
 
+def test_thumbnail_copy_and_scores_equivariant_under_permutations():
+    # Per-channel quantisation, an elementwise fold with a permutation-
+    # invariant max, exact integer sums and a max over tokens: permuting q's
+    # and K's channels together permutes thumbnails, residuals, scales and
+    # reconstructed keys with them and leaves every block score bit-identical;
+    # shuffling the valid tokens inside each block leaves scales and scores
+    # unchanged.
+    T, cap = 64, 512
+    k = _rand_keys(28, cap=cap)
+    rng = np.random.default_rng(29)
+    q = to_bf16(rng.standard_normal((2, 8, D)).astype(np.float32))
+    lengths = np.array([512, 237], np.int32)
+    thumb, resid, scales = oracle.quantize_keys_tr(k, lengths, T)
+    sc = oracle.block_scores_tr(q, thumb, scales, lengths, T)
+    khat = oracle.reconstruct_keys_tr(thumb, resid, scales, lengths, T)
+    perm = rng.permutation(D)
+    thumb_c, resid_c, scales_c = oracle.quantize_keys_tr(np.ascontiguousarray(k[..., perm]), lengths, T)
+    assert np.array_equal(scales_c, scales[..., perm])
+    assert np.array_equal(_thumb_codes(thumb_c), _thumb_codes(thumb)[..., perm])
+    assert np.array_equal(resid_c, resid[..., perm])
+    assert np.array_equal(oracle.reconstruct_keys_tr(thumb_c, resid_c, scales_c, lengths, T),
+                          khat[..., perm])
+    sc_c = oracle.block_scores_tr(np.ascontiguousarray(q[..., perm]), thumb_c, scales_c, lengths, T)
+    assert np.array_equal(sc_c, sc)
+    k_t = k.copy()
+    for b in range(k.shape[0]):
+        n = int(lengths[b])
+        for j0 in range(0, n, T):
+            idx = np.arange(j0, min(j0 + T, n))
+            k_t[b, :, idx] = k[b, :, rng.permutation(idx)]
+    thumb_t, _, scales_t = oracle.quantize_keys_tr(k_t, lengths, T)
+    assert np.array_equal(scales_t, scales)
+    assert np.array_equal(oracle.block_scores_tr(q, thumb_t, scales_t, lengths, T), sc)
+
+
 @pytest.mark.parametrize("delta", [math.inf, 1.0])
 def test_decode_tr_on_exact_keys_equals_library_attention(delta):
     # keys on the half-scale grid are reconstructed exactly, so the computer
