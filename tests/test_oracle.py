@@ -387,6 +387,32 @@ def test_scores_equivariant_under_channel_and_token_permutations():
     assert np.array_equal(oracle.block_scores(q, packed_t, scales_t, lengths, T), sc)
 
 
+def test_power_of_two_scaling_carries_through_copy_scores_and_selection():
+    # Scaling K (or q) by 2^e is exact in bf16 and commutes with every
+    # rounding of the quantiser and the fold: the int4 codes and the int8
+    # query stay the same, the scales (or the fold's a) gain 2^e, so every
+    # block score is multiplied by exactly 2^e, and the Top-delta selection
+    # with delta 2^e equals the original one.  (A fold that ignored the scales
+    # or a score factor without a, for example, breaks it.)
+    w, inp = _rand_case(31, B=2, G=4, Hkv=2, cap=512, lo=70, hi=512)
+    T, S = w.block_size, 3
+    q, k, lengths = inp["q"], inp["k"], inp["lengths"]
+    packed, scales = oracle.quantize_keys(k, lengths, T)
+    sc = oracle.block_scores(q, packed, scales, lengths, T)
+    _, mask = oracle.select(sc, lengths, w.num_kv_heads, w.capacity, T, S, 1.5)
+    for ek, eq in [(3, 0), (-4, 0), (0, 5), (2, -3)]:
+        k2 = to_bf16((from_bf16(k) * np.float32(2.0**ek)).astype(np.float32))
+        q2 = to_bf16((from_bf16(q) * np.float32(2.0**eq)).astype(np.float32))
+        packed2, scales2 = oracle.quantize_keys(k2, lengths, T)
+        assert np.array_equal(packed2, packed)
+        assert np.array_equal(from_bf16(scales2), from_bf16(scales) * np.float32(2.0**ek))
+        sc2 = oracle.block_scores(q2, packed2, scales2, lengths, T)
+        assert np.array_equal(sc2, sc * np.float32(2.0**(ek + eq)))
+        _, mask2 = oracle.select(sc2, lengths, w.num_kv_heads, w.capacity, T, S,
+                                 1.5 * 2.0**(ek + eq))
+        assert np.array_equal(mask2, mask)
+
+
 # ---------------------------------------------------------------- selection --
 
 def _read_golden():

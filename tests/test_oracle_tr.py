@@ -254,6 +254,31 @@ def _sdpa(q, k64, v, lengths, G, token_keep=None):
     return out
 
 
+def test_power_of_two_scaling_carries_through_thumbnails_and_scores():
+    # bf16(amax / 1.5) and k / s commute with a 2^e scaling of K, so the
+    # thumbnails and residuals stay the same, the scales and the reconstructed
+    # keys gain 2^e, and every thumbnail block score (with q scaled as well)
+    # is multiplied by exactly 2^(e_k + e_q).
+    T, cap = 64, 512
+    k = _rand_keys(30, cap=cap)
+    rng = np.random.default_rng(31)
+    q = to_bf16(rng.standard_normal((2, 8, D)).astype(np.float32))
+    lengths = np.array([512, 190], np.int32)
+    thumb, resid, scales = oracle.quantize_keys_tr(k, lengths, T)
+    sc = oracle.block_scores_tr(q, thumb, scales, lengths, T)
+    khat = oracle.reconstruct_keys_tr(thumb, resid, scales, lengths, T)
+    for ek, eq in [(4, 0), (-3, 2)]:
+        k2 = to_bf16((from_bf16(k) * np.float32(2.0**ek)).astype(np.float32))
+        q2 = to_bf16((from_bf16(q) * np.float32(2.0**eq)).astype(np.float32))
+        thumb2, resid2, scales2 = oracle.quantize_keys_tr(k2, lengths, T)
+        assert np.array_equal(thumb2, thumb) and np.array_equal(resid2, resid)
+        assert np.array_equal(from_bf16(scales2), from_bf16(scales) * np.float32(2.0**ek))
+        khat2 = oracle.reconstruct_keys_tr(thumb2, resid2, scales2, lengths, T)
+        assert np.array_equal(khat2, khat * 2.0**ek)
+        sc2 = oracle.block_scores_tr(q2, thumb2, scales2, lengths, T)
+        assert np.array_equal(sc2, sc * np.float32(2.0**(ek + eq)))
+
+
 def test_thumbnail_copy_and_scores_equivariant_under_permutations():
     # Per-channel quantisation, an elementwise fold with a permutation-
     # invariant max, exact integer sums and a max over tokens: permuting q's
