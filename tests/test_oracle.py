@@ -413,6 +413,47 @@ def test_power_of_two_scaling_carries_through_copy_scores_and_selection():
         assert np.array_equal(mask2, mask)
 
 
+@pytest.mark.parametrize("G,T", [(1, 128), (2, 64), (8, 128)])
+def test_other_group_and_block_sizes(G, T):
+    # The pins above mostly run G = 4, T = 64; the GPU path also serves
+    # G in {1, 2, 8} and T = 128 (the 256K workload).  Re-check the defining
+    # facts there: dense and masked attention against torch SDPA, the int4
+    # copy's half-step bound and scale rule, and the block-score bound.
+    w, inp = _rand_case(40 + G, B=2, G=G, Hkv=2, cap=1024, T=T, S=3, lo=150, hi=1024)
+    q, k, v, lengths = inp["q"], inp["k"], inp["v"], inp["lengths"]
+    out, mask, _ = oracle.decode(q, k, v, None, None, lengths, T, w.split_blocks, float("inf"))
+    np.testing.assert_allclose(out, _library_attention(q, k, v, lengths), rtol=0, atol=1e-10)
+    packed, scales = oracle.quantize_keys(k, lengths, T)
+    codes = _unpack_codes(packed)
+    sc = oracle.block_scores(q, packed, scales, lengths, T)
+    for b in range(w.batch):
+        n = int(lengths[b])
+        nb = -(-n // T)
+        for g in range(w.num_kv_heads):
+            kf = from_bf16(k[b, g, :n]).astype(np.float64)
+            sf = np.repeat(from_bf16(scales[b, g, :nb]).astype(np.float64), T, axis=0)[:n]
+            kc = codes[b, g, :n]
+            assert np.abs(kc).max() <= 7
+            assert (np.abs(kf - sf * kc) <= sf / 2 * (1 + 1e-6) + 1e-30).all()
+            assert (codes[b, g, n:nb * T] == 0).all()
+            for j in range(nb):
+                amax = np.abs(kf[j * T:(j + 1) * T]).max(axis=0)
+                sj = from_bf16(scales[b, g, j]).astype(np.float64)
+                assert (np.abs(sj - amax / 7) <= amax / 7 * 2.0**-8).all()
+        for h in range(w.num_q_heads):
+            g = h // G
+            qh = from_bf16(q[b, h]).astype(np.float64)
+            for j in range(nb):
+                sj = from_bf16(scales[b, g, j]).astype(np.float64)
+                kc = codes[b, g, j * T:min((j + 1) * T, n)]
+                exact = (kc * sj) @ qh / math.sqrt(D)
+                bound = np.abs(qh * sj).max() / 254 * np.abs(kc).sum(axis=1).max() / math.sqrt(D)
+                assert abs(sc[b, h, j] - exact.max()) <= bound * (1 + 1e-5) + 1e-6
+    out_s, mask_s, _ = oracle.decode(q, k, v, packed, scales, lengths, T, w.split_blocks, 1.0)
+    keep = _token_keep(mask_s, T, w.capacity)
+    np.testing.assert_allclose(out_s, _library_attention(q, k, v, lengths, keep), rtol=0, atol=1e-10)
+
+
 # ---------------------------------------------------------------- selection --
 
 def _read_golden():

@@ -362,6 +362,44 @@ def test_attend_tr_is_attention_over_reconstructed_keys():
     assert np.abs(out_d - ref).max() < 2e-2
 
 
+@pytest.mark.parametrize("G,T", [(1, 128), (8, 128)])
+def test_block_size_128_and_other_group_sizes(G, T):
+    # the pins above run T = 64; the GPU path also serves T = 128 and every G
+    cap = 1024
+    k = _rand_keys(40 + G, cap=cap)
+    rng = np.random.default_rng(41 + G)
+    v = to_bf16(rng.standard_normal((2, 2, cap, D)).astype(np.float32))
+    q = to_bf16(rng.standard_normal((2, 2 * G, D)).astype(np.float32))
+    lengths = np.array([1024, 333], np.int32)
+    thumb, resid, scales = oracle.quantize_keys_tr(k, lengths, T)
+    khat = oracle.reconstruct_keys_tr(thumb, resid, scales, lengths, T)
+    u = _thumb_codes(thumb)
+    sc = oracle.block_scores_tr(q, thumb, scales, lengths, T)
+    for b in range(2):
+        n = int(lengths[b])
+        nb = -(-n // T)
+        for g in range(2):
+            kf = from_bf16(k[b, g, :n]).astype(np.float64)
+            sf = np.repeat(from_bf16(scales[b, g, :nb]).astype(np.float64), T, axis=0)[:n]
+            assert (np.abs(kf - khat[b, g, :n]) <= sf / 508 * (1 + 1e-5) + 1e-30).all()
+            assert not thumb[b, g, n:nb * T].any() and not resid[b, g, n:nb * T].any()
+        for h in range(2 * G):
+            g = h // G
+            qh = from_bf16(q[b, h]).astype(np.float64)
+            for j in range(nb):
+                sj = from_bf16(scales[b, g, j]).astype(np.float64)
+                lv = 2 * u[b, g, j * T:min((j + 1) * T, n)] - 3
+                exact = (lv * sj / 2) @ qh / math.sqrt(D)
+                bound = np.abs(qh * sj).max() / 508 * np.abs(lv).sum(axis=1).max() / math.sqrt(D)
+                assert abs(sc[b, h, j] - exact.max()) <= bound * (1 + 1e-5) + 1e-6
+    words = oracle.mask_words(cap, T)
+    mask = rng.integers(0, 2**32, size=(2, 2, words), dtype=np.uint64).astype(np.uint32)
+    out, _ = oracle.attend_tr(q, thumb, resid, scales, v, lengths, mask, T)
+    keep = [np.stack([np.repeat(oracle.mask_to_blocks(mask[b, g], cap // T), T) for g in range(2)])
+            for b in range(2)]
+    assert np.abs(out - _sdpa(q, khat, v, lengths, G, keep)).max() < 1e-9
+
+
 def test_decode_tr_mask_follows_thumbnail_scores():
     # the step's mask is the Top-delta selection (pinned by enumeration in the
     # int4 tests) applied to the thumbnail scores, for both references
