@@ -23,6 +23,11 @@ _lib = None
 
 OK, BAD_ARG, BAD_LENGTH = 0, 1, 2
 
+# Reference maximum of the Top-delta filter (ffd_oracle.c, select_ref):
+RUNNING_MAX = 0        # running maximum inside each split (R5)
+PSEUDO_MAX_SEEDED = 1  # running maximum started at the sink/local pseudo-max (R15)
+PSEUDO_MAX_FIXED = 2   # the pages' rule: s_j >= pseudo-max - delta, fixed threshold (R15, R19)
+
 
 class OracleError(RuntimeError):
     pass
@@ -57,6 +62,9 @@ def _load():
                                         ctypes.c_float, p, p, p]
             lib.ffdo_decode_pseudo_max.argtypes = lib.ffdo_decode.argtypes
             lib.ffdo_select_pseudo_max.argtypes = lib.ffdo_select.argtypes
+            lib.ffdo_select_pseudo_max_fixed.argtypes = lib.ffdo_select.argtypes
+            lib.ffdo_decode_ref.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p,
+                                            ctypes.c_float, i, p, p, p]
             lib.ffdo_quantize_keys_tr.argtypes = [i, i, i, i, i, p, p, i, p, p, p]
             lib.ffdo_fold_query_tr.argtypes = [i, p, p, p, p]
             lib.ffdo_fold_query_tr.restype = None
@@ -123,17 +131,28 @@ def block_scores(q, packed, scales, lengths, block_size):
     return out
 
 
+def _reference(pseudo_max, reference):
+    if reference is None:
+        return PSEUDO_MAX_SEEDED if pseudo_max else RUNNING_MAX
+    if reference not in (RUNNING_MAX, PSEUDO_MAX_SEEDED, PSEUDO_MAX_FIXED):
+        raise OracleError(f"unknown reference {reference!r}")
+    return reference
+
+
 def select(scores, lengths, num_kv_heads, capacity, block_size, split_blocks, delta,
-           pseudo_max=False):
+           pseudo_max=False, reference=None):
     """Returns (keep [B,Hq,nblk] uint8, mask [B,Hkv,words] uint32).  pseudo_max
-    selects the sink/local reference maximum instead of starting each split's
-    running maximum at minus infinity."""
+    selects the seeded sink/local reference maximum instead of starting each
+    split's running maximum at minus infinity; ``reference`` (RUNNING_MAX,
+    PSEUDO_MAX_SEEDED, PSEUDO_MAX_FIXED) overrides it."""
+    ref = _reference(pseudo_max, reference)
     scores = _c(scores, np.float32)
     lengths = _c(lengths, np.int32)
     B, Hq, nblk = scores.shape
     keep = np.zeros((B, Hq, nblk), dtype=np.uint8)
     mask = np.zeros((B, num_kv_heads, mask_words(capacity, block_size)), dtype=np.uint32)
-    fn = _load().ffdo_select_pseudo_max if pseudo_max else _load().ffdo_select
+    fn = {RUNNING_MAX: _load().ffdo_select, PSEUDO_MAX_SEEDED: _load().ffdo_select_pseudo_max,
+          PSEUDO_MAX_FIXED: _load().ffdo_select_pseudo_max_fixed}[ref]
     _check(fn(B, Hq, num_kv_heads, capacity, block_size, split_blocks, _ptr(scores), _ptr(lengths),
               float(delta), _ptr(keep), _ptr(mask)))
     return keep, mask
@@ -155,8 +174,11 @@ def attend(q, k, v, lengths, mask, block_size):
     return out, lse
 
 
-def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta, pseudo_max=False):
-    """The whole step.  Returns (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores)."""
+def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta, pseudo_max=False,
+           reference=None):
+    """The whole step.  Returns (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores).
+    Reference maximum as ``select``."""
+    ref = _reference(pseudo_max, reference)
     q = _c(q, np.uint16)
     k = _c(k, np.uint16)
     v = _c(v, np.uint16)
@@ -168,10 +190,9 @@ def decode(q, k, v, packed, scales, lengths, block_size, split_blocks, delta, ps
     out = np.zeros((B, Hq, D), dtype=np.float64)
     mask = np.zeros((B, Hkv, mask_words(cap, block_size)), dtype=np.uint32)
     scores = np.zeros((B, Hq, cap // block_size), dtype=np.float32)
-    fn = _load().ffdo_decode_pseudo_max if pseudo_max else _load().ffdo_decode
-    _check(fn(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(k), _ptr(v),
-              _ptr(packed), _ptr(scales), _ptr(lengths), float(delta), _ptr(out), _ptr(mask),
-              _ptr(scores)))
+    _check(_load().ffdo_decode_ref(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(k),
+                                   _ptr(v), _ptr(packed), _ptr(scales), _ptr(lengths), float(delta),
+                                   ref, _ptr(out), _ptr(mask), _ptr(scores)))
     return out, mask, scores
 
 
@@ -258,9 +279,11 @@ def attend_tr(q, thumb, resid, scales, v, lengths, mask, block_size):
 
 
 def decode_tr(q, v, thumb, resid, scales, lengths, block_size, split_blocks, delta,
-              pseudo_max=False):
+              pseudo_max=False, reference=None):
     """The whole step on the thumbnail + residual format.  Returns
-    (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores)."""
+    (out [B,Hq,D] f64, mask [B,Hkv,words] u32, scores).  Reference maximum as
+    ``select``."""
+    ref = _reference(pseudo_max, reference)
     q = _c(q, np.uint16)
     v = _c(v, np.uint16)
     thumb = _c(thumb, np.uint8)
@@ -274,6 +297,6 @@ def decode_tr(q, v, thumb, resid, scales, lengths, block_size, split_blocks, del
     scores = np.zeros((B, Hq, cap // block_size), dtype=np.float32)
     _check(_load().ffdo_decode_tr(B, Hq, Hkv, cap, D, block_size, split_blocks, _ptr(q), _ptr(v),
                                   _ptr(thumb), _ptr(resid), _ptr(scales), _ptr(lengths),
-                                  float(delta), 1 if pseudo_max else 0, _ptr(out), _ptr(mask),
+                                  float(delta), ref, _ptr(out), _ptr(mask),
                                   _ptr(scores)))
     return out, mask, scores

@@ -29,9 +29,15 @@
  *   R7  the query is the last token: no causal mask; tokens >= length never
  *       contribute.
  *   R13 a sequence of length 0 yields a zero output row and an empty mask.
- *   R15 pseudo-max reference (optional mode): the sink tokens are block 0,
- *       the local tokens the last block; the split's running maximum starts
- *       at the larger of their two block scores.
+ *   R15 pseudo-max reference (optional modes): the sink tokens are block 0,
+ *       the local tokens the last block; the pseudo-max m~ is the larger of
+ *       their two block scores.
+ *   R19 the pages' rule with the pseudo-max: block j is kept iff
+ *       s_j >= m~ - delta, one fixed threshold per head for the whole
+ *       sequence.  A second variant, the seeded running maximum, starts each
+ *       split's running maximum at m~ and keeps updating it inside the split
+ *       (the build plan's reading of "pseudo-max seeding"); it keeps a subset
+ *       of the fixed rule's blocks.
  *   R16 thumbnail + residual key format (optional, the pages' own split of
  *       the K cache): per block and channel s = bf16(amax / 1.5); 2-bit code
  *       u = clamp(floor(k / s) + 2, 0, 3) naming the level (u - 1.5) s;
@@ -310,6 +316,45 @@ int ffdo_select_pseudo_max(int B, int Hq, int Hkv, int cap, int T, int S, const 
   return FFDO_OK;
 }
 
+/* ---- step 4'': Top-delta with the pseudo-max as a fixed threshold
+ *      (gist.science, Methodology 2, "Mechanism": keep j iff
+ *      s_j >= m~ - delta, where m~ is the pseudo-max of "Pseudo-Max
+ *      Approximation", estimated from the sink and the local tokens; R15,
+ *      R19) ----------------------------------------------------------------
+ * Per head h, mt_h = max(s_{0,h}, s_{nb-1,h}) and block j is kept for h iff
+ * s_{j,h} >= mt_h - delta (fp32 subtraction, inclusive comparison).  The
+ * threshold does not depend on the split, so the split size S has no effect
+ * on the result; a split may keep nothing. */
+int ffdo_select_pseudo_max_fixed(int B, int Hq, int Hkv, int cap, int T, int S,
+                                 const float *scores, const int32_t *lengths, float delta,
+                                 uint8_t *keep, uint32_t *mask) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || T <= 0 || cap % T != 0 || S <= 0)
+    return FFDO_BAD_ARG;
+  if (!(delta >= 0.0f)) return FFDO_BAD_ARG;
+  int G = Hq / Hkv, nblk = cap / T, words = (nblk + 31) / 32;
+  for (int b = 0; b < B; ++b)
+    if (lengths[b] < 0 || lengths[b] > cap) return FFDO_BAD_LENGTH;
+  memset(mask, 0, sizeof(uint32_t) * (size_t)B * Hkv * words);
+  if (keep) memset(keep, 0, (size_t)B * Hq * nblk);
+  for (int b = 0; b < B; ++b) {
+    int nb = (lengths[b] + T - 1) / T;
+    if (nb == 0) continue;
+    for (int h = 0; h < Hq; ++h) {
+      int g = h / G;
+      const float *s = scores + ((size_t)b * Hq + h) * nblk;
+      uint32_t *m = mask + ((size_t)b * Hkv + g) * words;
+      float pseudo = fmaxf(s[0], s[nb - 1]);
+      float threshold = pseudo - delta;
+      for (int j = 0; j < nb; ++j) {
+        int k = s[j] >= threshold;
+        if (keep) keep[((size_t)b * Hq + h) * nblk + j] = (uint8_t)k;
+        if (k) m[j / 32] |= 1u << (j % 32);
+      }
+    }
+  }
+  return FFDO_OK;
+}
+
 /* ---- step 5: exact attention over the selected blocks (gist.science,
  *      Methodology 3, stage "Fine-Grained Refinement"; R6, R7), fp64 -------- */
 
@@ -400,7 +445,21 @@ int ffdo_attend(int B, int Hq, int Hkv, int cap, int D, int T,
 static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
-                       float delta, double *out, uint32_t *mask, float *scores, int pseudo_max);
+                       float delta, double *out, uint32_t *mask, float *scores, int reference);
+
+/* Reference maximum of the Top-delta filter: 0 the running maximum inside each
+ * split (R5), 1 the running maximum seeded with the pseudo-max (R15), 2 the
+ * pseudo-max as a fixed threshold (R15, R19). */
+static int select_ref(int reference, int B, int Hq, int Hkv, int cap, int T, int S,
+                      const float *scores, const int32_t *lengths, float delta, uint32_t *mask) {
+  if (reference == 1)
+    return ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  if (reference == 2)
+    return ffdo_select_pseudo_max_fixed(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  if (reference == 0)
+    return ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  return FFDO_BAD_ARG;
+}
 
 int ffdo_decode(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                 const uint16_t *q, const uint16_t *k, const uint16_t *v,
@@ -410,7 +469,7 @@ int ffdo_decode(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                      mask, scores, 0);
 }
 
-/* The whole step with the pseudo-max reference (R15). */
+/* The whole step with the seeded pseudo-max reference (R15). */
 int ffdo_decode_pseudo_max(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                            const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
@@ -419,13 +478,22 @@ int ffdo_decode_pseudo_max(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                      mask, scores, 1);
 }
 
+/* The whole step with a chosen reference maximum (0, 1, 2 as select_ref). */
+int ffdo_decode_ref(int B, int Hq, int Hkv, int cap, int D, int T, int S,
+                    const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
+                    float delta, int reference, double *out, uint32_t *mask, float *scores) {
+  return decode_impl(B, Hq, Hkv, cap, D, T, S, q, k, v, packed, scales, lengths, delta, out,
+                     mask, scores, reference);
+}
+
 static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const uint8_t *packed, const uint16_t *scales, const int32_t *lengths,
-                       float delta, double *out, uint32_t *mask, float *scores, int pseudo_max) {
+                       float delta, double *out, uint32_t *mask, float *scores, int reference) {
   int rc = check_shape(B, Hq, Hkv, cap, D, T);
   if (rc != FFDO_OK) return rc;
-  if (S <= 0 || !(delta >= 0.0f)) return FFDO_BAD_ARG;
+  if (S <= 0 || !(delta >= 0.0f) || reference < 0 || reference > 2) return FFDO_BAD_ARG;
   int nblk = cap / T;
   float *own = NULL;
   if (!scores) {
@@ -441,9 +509,7 @@ static int decode_impl(int B, int Hq, int Hkv, int cap, int D, int T, int S,
     rc = ffdo_block_scores(B, Hq, Hkv, cap, D, T, q, packed, scales, lengths, scores);
     if (rc != FFDO_OK) { free(own); return rc; }
   }
-  rc = pseudo_max
-           ? ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask)
-           : ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  rc = select_ref(reference, B, Hq, Hkv, cap, T, S, scores, lengths, delta, mask);
   if (rc == FFDO_OK) rc = ffdo_attend(B, Hq, Hkv, cap, D, T, q, k, v, lengths, mask, out, NULL);
   free(own);
   return rc;
@@ -623,7 +689,8 @@ int ffdo_attend_tr(int B, int Hq, int Hkv, int cap, int D, int T, const uint16_t
 }
 
 /* The whole step on the thumbnail + residual format: thumbnail scores ->
- * Top-delta (running max, or the pseudo-max of R15 when pseudo_max != 0) ->
+ * Top-delta (pseudo_max: 0 the running max, 1 the seeded pseudo-max of R15,
+ * 2 the fixed pseudo-max threshold of R19) ->
  * attention with reconstructed keys.  delta = +INF selects every valid block. */
 int ffdo_decode_tr(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                    const uint16_t *q, const uint16_t *v, const uint8_t *thumb,
@@ -631,7 +698,7 @@ int ffdo_decode_tr(int B, int Hq, int Hkv, int cap, int D, int T, int S,
                    float delta, int pseudo_max, double *out, uint32_t *mask, float *scores) {
   int rc = check_shape(B, Hq, Hkv, cap, D, T);
   if (rc != FFDO_OK) return rc;
-  if (S <= 0 || !(delta >= 0.0f)) return FFDO_BAD_ARG;
+  if (S <= 0 || !(delta >= 0.0f) || pseudo_max < 0 || pseudo_max > 2) return FFDO_BAD_ARG;
   int nblk = cap / T;
   float *own = NULL;
   if (!scores) {
@@ -647,9 +714,7 @@ int ffdo_decode_tr(int B, int Hq, int Hkv, int cap, int D, int T, int S,
     rc = ffdo_block_scores_tr(B, Hq, Hkv, cap, D, T, q, thumb, scales, lengths, scores);
     if (rc != FFDO_OK) { free(own); return rc; }
   }
-  rc = pseudo_max
-           ? ffdo_select_pseudo_max(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask)
-           : ffdo_select(B, Hq, Hkv, cap, T, S, scores, lengths, delta, NULL, mask);
+  rc = select_ref(pseudo_max, B, Hq, Hkv, cap, T, S, scores, lengths, delta, mask);
   if (rc == FFDO_OK)
     rc = ffdo_attend_tr(B, Hq, Hkv, cap, D, T, q, thumb, resid, scales, v, lengths, mask, out, NULL);
   free(own);

@@ -755,6 +755,130 @@ def test_decode_pseudo_max_attends_over_its_mask():
         np.testing.assert_allclose(out, ref, atol=1e-10)
 
 
+# ------------------------- the pages' rule: pseudo-max as a fixed threshold --
+
+def _golden_examples(name):
+    """Parse a golden file of 'example' sections: meta lines and case lines."""
+    examples = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            if key == "example":
+                examples.append({"meta": {}, "cases": []})
+            elif key == "case":
+                examples[-1]["cases"].append(dict(item.split("=") for item in rest))
+            else:
+                examples[-1]["meta"][key] = rest
+    return examples
+
+
+_REFS = {"running": oracle.RUNNING_MAX, "seeded": oracle.PSEUDO_MAX_SEEDED,
+         "fixed": oracle.PSEUDO_MAX_FIXED}
+
+
+def test_select_pseudo_max_fixed_hand_worked_examples():
+    examples = _golden_examples("topdelta_pseudo_max_fixed_example.txt")
+    assert len(examples) == 2 and sum(len(e["cases"]) for e in examples) == 13
+    for ex in examples:
+        meta = ex["meta"]
+        T, nb = int(meta["block_size"][0]), int(meta["num_blocks"][0])
+        scores = np.array([[list(map(float, meta["scores_head0"]))]], np.float32)
+        lengths = np.array([nb * T], np.int32)
+        for case in ex["cases"]:
+            _, mask = oracle.select(scores, lengths, 1, nb * T, T, int(case["split"]),
+                                    float(case["delta"]), reference=_REFS[case["reference"]])
+            assert int(mask[0, 0, 0]) == int(case["mask"], 16), case
+
+
+def _declarative_keep_fixed(s, nb, delta):
+    """keep_j <=> s_j >= max(s_0, s_{nb-1}) - delta (fp32 subtraction)."""
+    thr = np.float32(np.float32(max(s[0], s[nb - 1])) - np.float32(delta))
+    return np.array([s[j] >= thr for j in range(nb)], bool)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_pseudo_max_fixed_matches_bruteforce_enumeration(seed):
+    rng = np.random.default_rng(500 + seed)
+    for _ in range(8):
+        nb = int(rng.integers(1, 13))
+        S = int(rng.choice([1, 3, 4, nb]))
+        G = int(rng.choice([1, 4]))
+        T = 64
+        scores = (rng.integers(-8, 9, size=(1, G, nb)) * 0.5).astype(np.float32)
+        delta = float(rng.choice([0.0, 0.5, 1.0, 2.5, np.inf]))
+        keep, mask = oracle.select(scores, np.array([nb * T], np.int32), 1, nb * T, T, S, delta,
+                                   reference=oracle.PSEUDO_MAX_FIXED)
+        got = oracle.mask_to_blocks(mask[0, 0], nb)
+        per_head = [_declarative_keep_fixed(scores[0, h], nb, delta) for h in range(G)]
+        satisfying = [np.array(bits) for bits in itertools.product([False, True], repeat=nb)
+                      if all(bits[j] == any(ph[j] for ph in per_head) for j in range(nb))]
+        assert len(satisfying) == 1 and np.array_equal(satisfying[0], got)
+        for h in range(G):
+            assert np.array_equal(keep[0, h, :nb].astype(bool), per_head[h])
+
+
+def test_select_pseudo_max_fixed_invariants():
+    rng = np.random.default_rng(41)
+    B, G, Hkv, T, nblk = 2, 4, 2, 64, 23
+    lengths = np.array([nblk * T, 9 * T + 3], np.int32)
+    scores = rng.standard_normal((B, G * Hkv, nblk)).astype(np.float32)
+    cap = nblk * T
+    prev = None
+    for d in [0.0, 0.25, 0.5, 1.0, 2.0, 4.0, np.inf]:
+        keep_f, mask_f = oracle.select(scores, lengths, Hkv, cap, T, 5, d,
+                                       reference=oracle.PSEUDO_MAX_FIXED)
+        _, mask_s = oracle.select(scores, lengths, Hkv, cap, T, 5, d,
+                                  reference=oracle.PSEUDO_MAX_SEEDED)
+
+        def blocks(m):
+            return np.array([[oracle.mask_to_blocks(m[b, g], nblk) for g in range(Hkv)]
+                             for b in range(B)])
+        fixed, seeded = blocks(mask_f), blocks(mask_s)
+        assert (seeded <= fixed).all()  # the seeded maximum never drops below the pseudo-max
+        for S in (1, 2, 7, nblk):  # no split enters the fixed rule
+            _, m2 = oracle.select(scores, lengths, Hkv, cap, T, S, d,
+                                  reference=oracle.PSEUDO_MAX_FIXED)
+            assert np.array_equal(m2, mask_f)
+        if prev is not None:
+            assert (prev <= fixed).all()  # monotone in delta
+        prev = fixed
+        for b in range(B):
+            nb = -(-int(lengths[b]) // T)
+            for h in range(G * Hkv):
+                mt = max(scores[b, h, 0], scores[b, h, nb - 1])
+                # every block at or above the pseudo-max is kept: the sink or
+                # local block that sets it in particular
+                assert keep_f[b, h, :nb][scores[b, h, :nb] >= mt].all()
+                assert not keep_f[b, h, nb:].any()
+            if d == np.inf:
+                assert fixed[b, :, :nb].all()
+        # the group union is the OR of the heads' own selections
+        for b in range(B):
+            for g in range(Hkv):
+                heads = keep_f[b, g * G:(g + 1) * G].astype(bool).any(axis=0)
+                assert np.array_equal(heads, fixed[b, g])
+
+
+def test_decode_pseudo_max_fixed_attends_over_its_mask():
+    w, inp = _rand_case(78, B=3, G=4, Hkv=2, cap=2048, T=64, S=4, lo=300, hi=2048)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+    for delta in (0.0, 1.0):
+        out, mask, sc2 = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales,
+                                       inp["lengths"], w.block_size, w.split_blocks, delta,
+                                       reference=oracle.PSEUDO_MAX_FIXED)
+        assert np.array_equal(sc2, sc)
+        _, want = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
+                                w.split_blocks, delta, reference=oracle.PSEUDO_MAX_FIXED)
+        assert np.array_equal(mask, want)
+        ref = _library_attention(inp["q"], inp["k"], inp["v"], inp["lengths"],
+                                 _token_keep(mask, w.block_size, w.capacity))
+        np.testing.assert_allclose(out, ref, atol=1e-10)
+
+
 def test_sparsity_adapts_to_attention_sharpness():
     # Methodology 2, Adaptivity (gist.science explainer): when attention is
     # concentrated, fewer blocks fall within delta of the peak.  Same queries,

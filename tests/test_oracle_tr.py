@@ -402,7 +402,7 @@ def test_block_size_128_and_other_group_sizes(G, T):
 
 def test_decode_tr_mask_follows_thumbnail_scores():
     # the step's mask is the Top-delta selection (pinned by enumeration in the
-    # int4 tests) applied to the thumbnail scores, for both references
+    # int4 tests) applied to the thumbnail scores, for every reference
     w = fw.random_small_workload(31, batch=3, group=4, num_kv_heads=2, capacity=1024,
                                  block_size=64, split_blocks=3, delta=2.0, lengths_lo=1,
                                  lengths_hi=1024, needles=1)
@@ -410,13 +410,13 @@ def test_decode_tr_mask_follows_thumbnail_scores():
     T = w.block_size
     thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], T)
     sc = oracle.block_scores_tr(inp["q"], thumb, scales, inp["lengths"], T)
-    for pseudo in (False, True):
+    for ref in (oracle.RUNNING_MAX, oracle.PSEUDO_MAX_SEEDED, oracle.PSEUDO_MAX_FIXED):
         for delta in (0.0, 1.5, 4.0):
             _, mask, sc2 = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales, inp["lengths"],
-                                            T, w.split_blocks, delta, pseudo)
+                                            T, w.split_blocks, delta, reference=ref)
             assert np.array_equal(sc2, sc)
             _, want = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, T,
-                                    w.split_blocks, delta, pseudo_max=pseudo)
+                                    w.split_blocks, delta, reference=ref)
             assert np.array_equal(mask, want)
 
 
