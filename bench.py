@@ -42,7 +42,7 @@ if ROOT not in sys.path:
 import ffd_workloads as fw  # noqa: E402
 
 DEFAULT_WORKLOAD = "long128k"
-REFERENCES = {"running": 0, "sink_local": 1}  # FFD_REFERENCE_* of include/ffd.h
+REFERENCES = {"running": 0, "sink_local": 1, "sink_local_fixed": 2}  # FFD_REFERENCE_* of include/ffd.h
 METRIC = "us per decode step (128K ctx) + effective HBM TB/s of the fused decode kernel"
 UNIT = "us/step"
 
@@ -1070,6 +1070,73 @@ def run_context_sweep(args):
     return 0
 
 
+def run_rho_sweep(args):
+    """The method's own regime: decode time against the kept fraction.  The
+    long-context shape with concentrated attention (ffd_workloads.RHO_DOMINANT:
+    flat keys, n of every 64 blocks raised by 6 logits, so the Top-delta rule
+    keeps n/64 of the blocks), the fused step timed from CUDA graphs for the
+    running maximum and the pages' fixed pseudo-max threshold, beside the same
+    kernel in dense mode.  Each row is checked against the oracle on the same
+    inputs (mask bit-exact, output max-abs / mean-abs), one JSON line."""
+    import torch
+    import oracle
+    from sparse_long_context_ffd_b200 import ffd
+    device = torch.device("cuda", torch.cuda.current_device())
+    l2 = getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 126 * 2**20)
+    peak, peak_src = load_peaks()
+    refs = [("running", ffd.FFD_REFERENCE_RUNNING_MAX), ("sink_local_fixed", ffd.FFD_REFERENCE_SINK_LOCAL_FIXED)]
+    rows = []
+    dense_us = None
+    for name in fw.RHO_DOMINANT:
+        w = fw.WORKLOADS[name]
+        inp = fw.make_inputs(w)
+        packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+        sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+        for ref_name, ref in refs:
+            probe = Replica(w, inp, device, 1)
+            probe.reference = ref
+            probe.step(0, w.delta)
+            torch.cuda.synchronize(device)
+            mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
+            out = probe.layers[0]["bufs"].out.float().cpu().numpy().astype(np.float64)
+            kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+            _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
+                                         w.split_blocks, w.delta, reference=ref)
+            want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
+                                        w.block_size)
+            err = np.abs(out - want_out)
+            algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)["total"]
+            del probe
+            layers = max(1, min(64, math.ceil(3 * l2 / algo)))
+            rep = Replica(w, inp, device, layers)
+            rep.reference = ref
+            _, per, _ = time_graph_steps(rep, w.delta, min(args.steps, 400), args.warmup, 1, device)
+            if dense_us is None:
+                _, per_d, _ = time_graph_steps(rep, float("inf"), min(args.steps, 400), args.warmup, 1,
+                                               device)
+                dense_us = float(np.mean(per_d)) * 1e3
+            rep.check_flags()
+            us = float(np.mean(per)) * 1e3
+            rows.append({"workload": name, "reference": ref_name,
+                         "kept_fraction": kept_blocks / max(1, valid_blocks),
+                         "decode_us": us, "algorithmic_bytes": algo,
+                         "tbs": algo / (us * 1e-6) / 1e12, "frac": algo / (us * 1e-6) / 1e9 / peak,
+                         "dense_us": dense_us, "vs_dense": dense_us / us,
+                         "oracle": {"mask_equal": bool(np.array_equal(mask, want_mask)),
+                                    "max_abs": float(err.max()), "mean_abs": float(err.mean())}})
+            del rep
+            torch.cuda.empty_cache()
+        del inp, packed, scales, sc
+    line = {"mode": "rho-sweep", "metric": "us per decode launch vs kept fraction (128K)",
+            "unit": "us",
+            "workload": "long-context shape (B1 Hq32 Hkv8 D128 N131072 T64 S64 delta 3) with "
+                        "concentrated attention: keys 0.1 N(0,1), n of every 64 blocks raised by "
+                        "6 logits (ffd_workloads.RHO_DOMINANT)",
+            "peak_gbs": peak, "peak_source": peak_src, "rows": rows}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1083,8 +1150,9 @@ def main(argv=None):
     ap.add_argument("--clocks-csv", default=None,
                     help="also write the raw nvidia-smi clock samples of the timed window here")
     ap.add_argument("--reference", choices=sorted(REFERENCES), default="running",
-                    help="Top-delta reference maximum: running max in the split, or the "
-                         "pseudo-max of the sink and local blocks")
+                    help="Top-delta reference maximum: running max in the split, the running "
+                         "max seeded with the sink/local pseudo-max, or that pseudo-max as a "
+                         "fixed threshold")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1094,6 +1162,9 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=150.0)
     ap.add_argument("--context-sweep", action="store_true",
                     help="the long-context workload at 16K..256K tokens, sparse and dense (one line)")
+    ap.add_argument("--rho-sweep", action="store_true",
+                    help="the 128K shape with concentrated attention at kept fractions 1/64..1, "
+                         "running and fixed pseudo-max references, oracle-checked (one line)")
     ap.add_argument("--shards", type=int, default=0,
                     help="time one rank's share of a context-sharded step over this many shards")
     ap.add_argument("--profile-steps", type=int, default=0,
@@ -1111,6 +1182,8 @@ def main(argv=None):
         return run_shard_measure(args)
     if args.context_sweep:
         return run_context_sweep(args)
+    if args.rho_sweep:
+        return run_rho_sweep(args)
     return run_gpu(args)
 
 

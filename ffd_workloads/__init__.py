@@ -24,6 +24,14 @@ Recipe (all float work in fp32, one final round-to-nearest-even to bf16):
     key row of the block gets + 3 * q_h / |q_h|.
   * tokens at or beyond each sequence's length (the unused cache tail) hold
     finite poison values, so that a kernel that reads past the length fails.
+  * controlled sparsity (the "rho" family, the method's own regime of
+    concentrated attention): keys are key_scale * N(0, 1) (nearly flat scores)
+    and in every split of S blocks, aligned at block 0, `dominant_per_split`
+    blocks -- the split's first block and others drawn without replacement --
+    get every key row + margin * sqrt(D) * sum_h q_h / |q_h|^2 over the kv-head's
+    query heads h, which raises each head's logits by about `margin`; with
+    margin > delta plus the noise, the Top-delta rule keeps about
+    dominant_per_split / S of the blocks.
 """
 from __future__ import annotations
 
@@ -62,6 +70,9 @@ class Workload:
     drift_sigma: float = 0.0
     head_dim: int = HEAD_DIM
     description: str = ""
+    key_scale: float = 1.0  # standard deviation of the keys' N(0, 1) draw
+    dominant_per_split: Optional[int] = None  # raised blocks per split (rho family)
+    dominant_margin: float = 0.0  # logits added to those blocks' keys
 
     @property
     def group(self) -> int:
@@ -104,7 +115,30 @@ WORKLOADS: Dict[str, Workload] = {
 
 MAX256K_DELTAS = (1.0, 2.0, 3.0, 4.0, float("inf"))
 
+# Controlled sparsity on the long-context shape: raised blocks per split of 64
+# and the kept fraction they give (1/64, ~0.05, 0.25, 0.5, 1).
+RHO_DOMINANT = {"rho1of64": 1, "rho0p05": 3, "rho0p25": 16, "rho0p5": 32, "rho1": 64}
+
+
+def rho_workload(name: str) -> Workload:
+    """The long-context shape (B1 Hq32 Hkv8 N131072 T64 S64 delta 3) with
+    concentrated attention: flat keys (0.1 N(0, 1)) and RHO_DOMINANT[name]
+    blocks per split raised by 6 logits."""
+    n = RHO_DOMINANT[name]
+    return Workload(
+        name=name, batch=1, num_q_heads=32, num_kv_heads=8, capacity=131072, block_size=64,
+        split_blocks=64, delta=3.0, seed=20 + sorted(RHO_DOMINANT).index(name), context=131072,
+        needles=0, key_scale=0.1, dominant_per_split=n, dominant_margin=6.0,
+        description=(f"long-context shape with concentrated attention: B1 Hq32 Hkv8 D128 N131072 "
+                     f"T64 S64 delta3, keys 0.1 N(0,1), {n} of every 64 blocks raised by 6 "
+                     f"logits (kept fraction ~{n / 64:.3g})"))
+
+
+for _name in RHO_DOMINANT:
+    WORKLOADS[_name] = rho_workload(_name)
+
 _STREAM_Q, _STREAM_K, _STREAM_V, _STREAM_DRIFT, _STREAM_META = 1, 2, 3, 4, 5
+_STREAM_DOMINANT = 6
 
 
 def _rng(seed: int, stream: int, b: int = 0, g: int = 0) -> np.random.Generator:
@@ -182,6 +216,24 @@ def make_inputs(w: Workload, lengths: Optional[np.ndarray] = None,
         b, g = bg
         n = int(lengths[b])
         kk = _rng(w.seed, _STREAM_K, b, g).standard_normal((n, D), dtype=np.float32)
+        if w.key_scale != 1.0:
+            kk *= np.float32(w.key_scale)
+        if w.dominant_per_split and n > 0:
+            T, S = w.block_size, w.split_blocks
+            qg = qf[b, g * G:(g + 1) * G]
+            bump = np.zeros(D, dtype=np.float32)
+            for h in range(G):
+                bump += qg[h] / np.sum(qg[h] * qg[h], dtype=np.float32)
+            bump *= np.float32(w.dominant_margin * np.sqrt(D))
+            rng_d = _rng(w.seed, _STREAM_DOMINANT, b, g)
+            nb = -(-n // T)
+            for j0 in range(0, nb, S):
+                width = min(S, nb - j0)
+                extra = min(w.dominant_per_split, width) - 1
+                picks = [0] + sorted((1 + rng_d.choice(width - 1, size=extra, replace=False)).tolist())
+                for j in picks:
+                    t0 = (j0 + j) * T
+                    kk[t0:min(t0 + T, n)] += bump
         if w.drift_sigma > 0.0 and n > 0:
             # random walk per channel, accumulated along the token axis
             steps = _rng(w.seed, _STREAM_DRIFT, b, g).standard_normal((D, n), dtype=np.float32)

@@ -168,19 +168,26 @@ ffd_status ffd_decode_step(const ffd_shape *shape, const void *q_bf16, const voi
                            void *workspace, size_t workspace_bytes, void *cuda_stream);
 
 /* Reference maximum of the Top-delta filter. */
-#define FFD_REFERENCE_RUNNING_MAX 0 /* running max inside each split (default) */
-#define FFD_REFERENCE_SINK_LOCAL 1  /* pseudo-max from the sink and local blocks */
+#define FFD_REFERENCE_RUNNING_MAX 0       /* running max inside each split (default) */
+#define FFD_REFERENCE_SINK_LOCAL 1        /* running max started at the sink/local pseudo-max */
+#define FFD_REFERENCE_SINK_LOCAL_FIXED 2  /* the sink/local pseudo-max as a fixed threshold */
 
 typedef struct {
   /* FFD_REFERENCE_RUNNING_MAX: each split's running maximum starts at -inf
    *   (the first block of every split is kept).
-   * FFD_REFERENCE_SINK_LOCAL: the pseudo-max of gist.science explainer,
-   *   Methodology 2 "Pseudo-Max Approximation" -- the reference maximum is
-   *   estimated from the sink tokens and the local tokens only.  Here: per
-   *   query head, mt = max(score of block 0, score of block nb - 1), and each
-   *   split's running maximum starts at mt.  Every split still decides on its
-   *   own (each CTA scores those two blocks itself); a split may keep nothing;
-   *   the head's highest-scoring block is always kept. */
+   * FFD_REFERENCE_SINK_LOCAL_FIXED: the rule of gist.science explainer,
+   *   Methodology 2 "Mechanism" with the pseudo-max of "Pseudo-Max
+   *   Approximation" (estimated from the sink tokens and the local tokens
+   *   only).  Per query head, mt = max(score of block 0, score of block
+   *   nb - 1), and block j is kept iff score_j >= mt - delta: one threshold
+   *   for the whole sequence, so the split size does not change the mask.
+   *   Every block at or above mt is kept; a split may keep nothing.
+   * FFD_REFERENCE_SINK_LOCAL: a seeded variant -- each split's running
+   *   maximum starts at mt and keeps rising inside the split as under
+   *   FFD_REFERENCE_RUNNING_MAX; it keeps a subset of the fixed rule's
+   *   blocks and the head's highest-scoring block is always kept.
+   * In both pseudo-max modes every split still decides on its own (each CTA
+   * scores the sink and local blocks itself); a split may keep nothing. */
   int32_t reference;
   /* 1: re-quantise each sequence's last block first, as ffd_decode_step. */
   int32_t requant_last;

@@ -254,7 +254,8 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
                          const void *v_new = nullptr, uint64_t wait_limit_ns = kWaitLimitNs) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
-  if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL)
+  if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL &&
+      reference != FFD_REFERENCE_SINK_LOCAL_FIXED)
     return FFD_ERR_INVALID_ARG;
   if (partials_only) {
     // a context shard: splits must not straddle shards, and the pseudo-max

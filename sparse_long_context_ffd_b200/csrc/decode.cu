@@ -625,24 +625,26 @@ __global__ void __launch_bounds__(kThreads, 2)
                              kHeadDim + 32 * t4,
                    SF::part(gid), qv);
     float run0 = -INFINITY, run1 = -INFINITY;  // running max of heads 2*t4, 2*t4 + 1
+    // the pages' rule: the pseudo-max is a fixed threshold (no running update)
+    const bool fixed_ref = p.reference == 2;
     int qn = 0;
     // the Top-delta decision for scan entry e
     auto decide = [&](int e, float s0, float s1) {
-      if (e < nref) {  // reference blocks: the split's running max starts at their max
+      if (e < nref) {  // reference blocks: the pseudo-max is their max
         run0 = fmaxf(run0, s0);
         run1 = fmaxf(run1, s1);
         return;
       }
       const int i = e - nref;
-      // Top-delta against the running maximum of the split, union over the group
+      // Top-delta against the reference maximum, union over the group
       bool keep = false;
       if (gid == 0) {
         if (2 * t4 < G) {
-          run0 = fmaxf(run0, s0);
+          if (!fixed_ref) run0 = fmaxf(run0, s0);
           keep = s0 >= __fsub_rn(run0, p.delta);
         }
         if (2 * t4 + 1 < G) {
-          run1 = fmaxf(run1, s1);
+          if (!fixed_ref) run1 = fmaxf(run1, s1);
           keep = keep || (s1 >= __fsub_rn(run1, p.delta));
         }
       }

@@ -47,8 +47,9 @@ struct DecodeParams {
   int32_t dense;
   // fused decode step: re-quantise each sequence's last key block first
   int32_t requant_last;
-  // reference maximum: 0 = running max inside the split, 1 = pseudo-max from
-  // the sink (first) and local (last) blocks
+  // reference maximum: 0 = running max inside the split, 1 = running max
+  // started at the pseudo-max of the sink (first) and local (last) blocks,
+  // 2 = that pseudo-max as a fixed threshold
   int32_t reference;
   const uint16_t *k;         // bf16 [B][Hkv][cap][D] (read by the re-quantisation)
   uint8_t *packed_out;       // = packed, written for the last block

@@ -41,7 +41,8 @@ EXPORTED = (
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
-FFD_REFERENCE_SINK_LOCAL = 1
+FFD_REFERENCE_SINK_LOCAL = 1        # running maximum started at the sink/local pseudo-max
+FFD_REFERENCE_SINK_LOCAL_FIXED = 2  # the sink/local pseudo-max as a fixed threshold
 
 # Size of the library's built-in scratch array used by ffd_decode_no_alloc.
 FFD_NO_ALLOC_SCRATCH_BYTES = 16 << 20

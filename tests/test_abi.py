@@ -121,7 +121,7 @@ def test_bad_arguments_rejected_on_host():
                                None) == ffd.FFD_ERR_INVALID_ARG
     assert lib.ffd_decode_step(ctypes.byref(s), a, a, a, a, a, a, -1.0, a, a, a, ws,
                                None) == ffd.FFD_ERR_INVALID_ARG
-    for bad in (ffd.DecodeOptions(2, 0), ffd.DecodeOptions(-1, 0), ffd.DecodeOptions(0, 2),
+    for bad in (ffd.DecodeOptions(3, 0), ffd.DecodeOptions(-1, 0), ffd.DecodeOptions(0, 2),
                 ffd.DecodeOptions(0, 0, -1)):
         assert lib.ffd_decode_ex(ctypes.byref(s), ctypes.byref(bad), a, a, a, a, a, a, 1.0, a, a,
                                  a, ws, None) == ffd.FFD_ERR_INVALID_ARG
@@ -162,10 +162,22 @@ def test_thumb_resid_arguments_rejected_on_host():
     s_bad = ffd.make_shape(2, 16, 4, 4096, 32, 16)
     assert q(ctypes.byref(s_bad), a, a, 0, a, a, a, None) == ffd.FFD_ERR_UNSUPPORTED
     assert ffd.thumb_bytes(s_bad) == 0 and ffd.residual_bytes(s_bad) == 0
-    # context shards: the pseudo-max is rejected as for the int4 format
-    sink = ffd.DecodeOptions(1, 0)
-    assert lib.ffd_decode_partials_tr(ctypes.byref(s), ctypes.byref(sink), a, a, a, a, a, a, a, 1.0,
-                                      a, ws, None) == ffd.FFD_ERR_UNSUPPORTED
+    # context shards: both pseudo-max modes are rejected as for the int4 format
+    for ref in (ffd.FFD_REFERENCE_SINK_LOCAL, ffd.FFD_REFERENCE_SINK_LOCAL_FIXED):
+        sink = ffd.DecodeOptions(ref, 0)
+        assert lib.ffd_decode_partials_tr(ctypes.byref(s), ctypes.byref(sink), a, a, a, a, a, a, a,
+                                          1.0, a, ws, None) == ffd.FFD_ERR_UNSUPPORTED
+
+
+def test_reference_codes_match_the_oracle_numbering():
+    # the parity tests pass FFD_REFERENCE_* straight to the oracle
+    import oracle
+    assert ffd.FFD_REFERENCE_RUNNING_MAX == oracle.RUNNING_MAX == 0
+    assert ffd.FFD_REFERENCE_SINK_LOCAL == oracle.PSEUDO_MAX_SEEDED == 1
+    assert ffd.FFD_REFERENCE_SINK_LOCAL_FIXED == oracle.PSEUDO_MAX_FIXED == 2
+    header = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                               "include", "ffd.h")).read()
+    assert "#define FFD_REFERENCE_SINK_LOCAL_FIXED 2" in header
 
 
 def test_append_arguments_rejected_on_host():
@@ -185,7 +197,7 @@ def test_append_arguments_rejected_on_host():
     for name in ("kn", "vn", "k", "v", "p", "sc"):
         assert app(**{name: None}) == ffd.FFD_ERR_INVALID_ARG, name
     assert app(kn=a + 4) == ffd.FFD_ERR_INVALID_ARG and app(vn=a + 2) == ffd.FFD_ERR_INVALID_ARG
-    assert app(ref=2) == ffd.FFD_ERR_INVALID_ARG
+    assert app(ref=3) == ffd.FFD_ERR_INVALID_ARG and app(ref=-1) == ffd.FFD_ERR_INVALID_ARG
     assert app(delta=float("nan")) == ffd.FFD_ERR_INVALID_ARG
     # the thumbnail form needs bf16 K here: the append writes it
     assert app_tr(k=None) == ffd.FFD_ERR_INVALID_ARG

@@ -101,14 +101,16 @@ def _run_case(w, inp, fmt, reference, delta, first_back=4, lengths_final=None):
 
 
 def _oracle(w, inp, fmt, reference, delta, lengths):
-    pseudo = reference == ffd.FFD_REFERENCE_SINK_LOCAL
+    # (FFD_REFERENCE_* and the oracle's reference codes share their numbering)
     T, S = w.block_size, w.split_blocks
     if fmt == "tr":
         th, re, sc = oracle.quantize_keys_tr(inp["k"], lengths, T)
-        out, mask, _ = oracle.decode_tr(inp["q"], inp["v"], th, re, sc, lengths, T, S, delta, pseudo)
+        out, mask, _ = oracle.decode_tr(inp["q"], inp["v"], th, re, sc, lengths, T, S, delta,
+                                        reference=reference)
     else:
         p, sc = oracle.quantize_keys(inp["k"], lengths, T)
-        out, mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], p, sc, lengths, T, S, delta, pseudo)
+        out, mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], p, sc, lengths, T, S, delta,
+                                     reference=reference)
     return out, mask
 
 
@@ -116,7 +118,7 @@ def _oracle(w, inp, fmt, reference, delta, lengths):
 @pytest.mark.parametrize("T,delta,reference", [
     (64, 2.0, ffd.FFD_REFERENCE_RUNNING_MAX), (128, 0.75, ffd.FFD_REFERENCE_RUNNING_MAX),
     (64, INF, ffd.FFD_REFERENCE_RUNNING_MAX), (64, 0.5, ffd.FFD_REFERENCE_SINK_LOCAL),
-    (128, 1.5, ffd.FFD_REFERENCE_SINK_LOCAL)])
+    (128, 1.5, ffd.FFD_REFERENCE_SINK_LOCAL), (64, 1.0, ffd.FFD_REFERENCE_SINK_LOCAL_FIXED)])
 def test_decode_append_equals_store_then_step(fmt, T, delta, reference):
     w = fw.random_small_workload(80 + T, 3, 4, 2, 32 * T, T, 3, 2.0, 12 * T, 32 * T, needles=2)
     inp = fw.make_inputs(w)

@@ -280,31 +280,41 @@ def test_decode_step_equals_quantize_then_decode(T, delta):
 
 
 # ------------------------------------- pseudo-max reference (sink + local) --
+# both pseudo-max modes: the running maximum seeded with the pseudo-max, and
+# the pages' fixed threshold (the library's FFD_REFERENCE_* and the oracle's
+# reference codes share their numbering)
+PSEUDO_REFS = [ffd.FFD_REFERENCE_SINK_LOCAL, ffd.FFD_REFERENCE_SINK_LOCAL_FIXED]
 
+
+def _ref_id(r):
+    return "fixed" if r == ffd.FFD_REFERENCE_SINK_LOCAL_FIXED else "seeded"
+
+
+@pytest.mark.parametrize("ref", PSEUDO_REFS, ids=_ref_id)
 @pytest.mark.parametrize("delta", [0.0, 0.75, 2.0, INF])
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c[0]}")
-def test_decode_pseudo_max_small(case, delta):
+def test_decode_pseudo_max_small(case, delta, ref):
     w, inp = _small(case)
     packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
     want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales,
                                            inp["lengths"], w.block_size, w.split_blocks, delta,
-                                           pseudo_max=True)
+                                           reference=ref)
     gc = GpuCase(w, inp)
     gc.quantize(0)
     ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
-                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace,
-                  reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace, reference=ref)
     torch.cuda.synchronize()
     from gpu_util import bf16_to_np_f32
     mask = gc.bufs.mask.cpu().numpy().view(np.uint32)
-    assert_mask_equal(mask, want_mask, f"pseudo case {case[0]} delta {delta}")
-    assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out,
-                        f"pseudo case {case[0]} delta {delta}")
+    tag = f"pseudo {_ref_id(ref)} case {case[0]} delta {delta}"
+    assert_mask_equal(mask, want_mask, tag)
+    assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, tag)
     assert ffd.check_device_status(gc.bufs.workspace) == 0
 
 
+@pytest.mark.parametrize("ref", PSEUDO_REFS, ids=_ref_id)
 @pytest.mark.parametrize("T,delta", [(64, 0.5), (128, 1.5)])
-def test_decode_step_pseudo_max_equals_quantize_then_decode(T, delta):
+def test_decode_step_pseudo_max_equals_quantize_then_decode(T, delta, ref):
     # several splits per sequence, so CTAs that do not own the last block
     # build its int4 tile themselves while the owner rewrites it
     w = fw.random_small_workload(60 + T, 3, 4, 2, 32 * T, T, 3, 2.0, 12 * T, 32 * T, needles=2)
@@ -319,12 +329,10 @@ def test_decode_step_pseudo_max_equals_quantize_then_decode(T, delta):
         a.lengths.copy_(ln)
         b.lengths.copy_(ln)
         ffd.decode_ex(a.shape, a.q, a.k, a.v, a.bufs.k_packed, a.bufs.k_scales, a.lengths, delta,
-                      a.bufs.out, a.bufs.mask, a.bufs.workspace,
-                      reference=ffd.FFD_REFERENCE_SINK_LOCAL, requant_last=True)
+                      a.bufs.out, a.bufs.mask, a.bufs.workspace, reference=ref, requant_last=True)
         b.quantize(ffd.FFD_LAST_BLOCK)
         ffd.decode_ex(b.shape, b.q, b.k, b.v, b.bufs.k_packed, b.bufs.k_scales, b.lengths, delta,
-                      b.bufs.out, b.bufs.mask, b.bufs.workspace,
-                      reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+                      b.bufs.out, b.bufs.mask, b.bufs.workspace, reference=ref)
         torch.cuda.synchronize()
         assert torch.equal(a.bufs.out.view(torch.int16), b.bufs.out.view(torch.int16))
         assert torch.equal(a.bufs.mask, b.bufs.mask)
@@ -332,34 +340,34 @@ def test_decode_step_pseudo_max_equals_quantize_then_decode(T, delta):
         assert torch.equal(a.bufs.k_scales.view(torch.int16), b.bufs.k_scales.view(torch.int16))
     packed, scales = oracle.quantize_keys(inp["k"], final, w.block_size)
     want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales, final,
-                                           w.block_size, w.split_blocks, delta, pseudo_max=True)
+                                           w.block_size, w.split_blocks, delta, reference=ref)
     from gpu_util import bf16_to_np_f32
     assert_mask_equal(a.bufs.mask.cpu().numpy().view(np.uint32), want_mask, "pseudo step")
     assert_output_close(bf16_to_np_f32(a.bufs.out).astype(np.float64), want_out, "pseudo step")
 
 
+@pytest.mark.parametrize("ref", PSEUDO_REFS, ids=_ref_id)
 @pytest.mark.parametrize("name,delta", [("long128k", 3.0), ("max256k", 1.0), ("ragged", 3.0)])
-def test_full_config_pseudo_max(name, delta):
+def test_full_config_pseudo_max(name, delta, ref):
     w = fw.WORKLOADS[name]
     inp = fw.make_inputs(w)
     packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
     sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
     _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
-                                 w.split_blocks, delta, pseudo_max=True)
+                                 w.split_blocks, delta, reference=ref)
     want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
                                 w.block_size)
     gc = GpuCase(w, inp)
     gc.quantize(0)
     ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
-                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace,
-                  reference=ffd.FFD_REFERENCE_SINK_LOCAL)
+                  delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace, reference=ref)
     torch.cuda.synchronize()
     from gpu_util import bf16_to_np_f32
     mask = gc.bufs.mask.cpu().numpy().view(np.uint32)
-    assert_mask_equal(mask, want_mask, f"{name} pseudo")
-    mx, mean = assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out,
-                                   f"{name} pseudo")
+    tag = f"{name} pseudo {_ref_id(ref)}"
+    assert_mask_equal(mask, want_mask, tag)
+    mx, mean = assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, tag)
     nblk = w.capacity // w.block_size
     kept = sum(int(oracle.mask_to_blocks(mask[b, g], nblk).sum())
                for b in range(w.batch) for g in range(w.num_kv_heads))
-    print(name, "pseudo-max kept", kept, "max-abs", mx, "mean-abs", mean)
+    print(tag, "kept", kept, "max-abs", mx, "mean-abs", mean)

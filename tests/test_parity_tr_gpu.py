@@ -157,19 +157,23 @@ def test_decode_tr_small(case, delta):
     assert ffd.check_device_status(tc.bufs.workspace) == 0
 
 
+@pytest.mark.parametrize("ref", [ffd.FFD_REFERENCE_SINK_LOCAL, ffd.FFD_REFERENCE_SINK_LOCAL_FIXED],
+                         ids=["seeded", "fixed"])
 @pytest.mark.parametrize("delta", [0.0, 1.0, 3.0])
 @pytest.mark.parametrize("case", SMALL[:6], ids=lambda c: f"s{c[0]}")
-def test_decode_tr_pseudo_max_small(case, delta):
+def test_decode_tr_pseudo_max_small(case, delta, ref):
+    # (the library's FFD_REFERENCE_* and the oracle's reference codes share
+    # their numbering)
     w, inp = _small(case)
     thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], w.block_size)
     want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales,
                                               inp["lengths"], w.block_size, w.split_blocks, delta,
-                                              pseudo_max=True)
+                                              reference=ref)
     tc = TrCase(w, inp)
     tc.quantize(0)
-    out, mask = tc.decode(delta, reference=ffd.FFD_REFERENCE_SINK_LOCAL)
-    assert_mask_equal(mask, want_mask, f"tr pseudo case {case[0]} delta {delta}")
-    assert_output_close(out, want_out, f"tr pseudo case {case[0]} delta {delta}")
+    out, mask = tc.decode(delta, reference=ref)
+    assert_mask_equal(mask, want_mask, f"tr pseudo {ref} case {case[0]} delta {delta}")
+    assert_output_close(out, want_out, f"tr pseudo {ref} case {case[0]} delta {delta}")
 
 
 @pytest.mark.parametrize("T", [64, 128])
@@ -220,7 +224,7 @@ def test_decode_tr_bad_lengths_flagged_and_graph_replay():
 @pytest.mark.parametrize("T,delta,reference", [
     (64, 2.0, ffd.FFD_REFERENCE_RUNNING_MAX), (128, 0.75, ffd.FFD_REFERENCE_RUNNING_MAX),
     (64, INF, ffd.FFD_REFERENCE_RUNNING_MAX), (64, 0.5, ffd.FFD_REFERENCE_SINK_LOCAL),
-    (128, 1.5, ffd.FFD_REFERENCE_SINK_LOCAL)])
+    (128, 1.5, ffd.FFD_REFERENCE_SINK_LOCAL), (64, 1.0, ffd.FFD_REFERENCE_SINK_LOCAL_FIXED)])
 def test_decode_tr_step_equals_quantize_then_decode(T, delta, reference):
     # several splits per sequence; decoding starts 4 tokens early and appends
     # one token per step, re-quantising the last block inside the launch
@@ -245,8 +249,7 @@ def test_decode_tr_step_equals_quantize_then_decode(T, delta, reference):
         assert torch.equal(a.bufs.k_scales.view(torch.int16), b.bufs.k_scales.view(torch.int16))
     thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], final, T)
     want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales, final, T,
-                                              w.split_blocks, delta,
-                                              pseudo_max=reference == ffd.FFD_REFERENCE_SINK_LOCAL)
+                                              w.split_blocks, delta, reference=reference)
     assert_mask_equal(a.bufs.mask.cpu().numpy().view(np.uint32), want_mask, "tr step")
     assert_output_close(bf16_to_np_f32(a.bufs.out).astype(np.float64), want_out, "tr step")
     assert ffd.check_device_status(a.bufs.workspace) == 0
