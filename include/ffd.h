@@ -366,15 +366,30 @@ ffd_status ffd_merge_partials(const ffd_shape *local_shape, int32_t num_shards, 
  * 16 MiB (16777216 bytes) return FFD_ERR_WORKSPACE before any launch.
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it, so make that first call before any stream
- * capture.  Every call clears the array's counters and error word on the
- * stream first; the array is shared by all calls on a device and keeps the
- * last call's contents, so calls that overlap on the GPU race and must be
- * serialised by the caller.  Device-side length errors still yield zero rows
- * and an empty mask, but there is no workspace from which to read the flag. */
+ * capture.  Every call that passes its host checks clears the array's
+ * counters and error word on the stream just before its launch (a rejected
+ * call writes nothing); the array is shared by all calls on a device and
+ * keeps the last call's contents, so calls that overlap on the GPU race and
+ * must be serialised by the caller.  Device-side errors are reported by
+ * ffd_no_alloc_device_status: a length outside [0, cap] (zero rows and an
+ * empty mask for that sequence), or a bounded wait that ran out (the output
+ * is then not valid).  Outside a stream capture each call looks the array's
+ * address up again, so it stays right after a device reset; inside a capture
+ * the address from the last call outside it is used. */
 ffd_status ffd_decode_no_alloc(const ffd_shape *shape, const void *q_bf16, const void *k_bf16,
                                const void *v_bf16, const void *k_packed, const void *k_scales,
                                const int32_t *d_lengths, float delta, void *out_bf16,
                                uint32_t *mask, void *cuda_stream);
+
+/* The error word of ffd_decode_no_alloc's built-in array on the current
+ * device, as ffd_check_device_status reads a workspace's: synchronise the
+ * stream, read the flags the last ffd_decode_no_alloc call on this device
+ * left and clear them.  Call it after that call and before the next one.
+ * Returns FFD_ERR_TIMEOUT if FFD_DEVICE_FLAG_TIMEOUT was set (that call's
+ * output is not valid), FFD_ERR_DEVICE_CHECK for any other flag,
+ * FFD_ERR_INVALID_ARG while the stream is being captured.  Allocates
+ * nothing; the paper has no counterpart. */
+ffd_status ffd_no_alloc_device_status(uint32_t *flags_out, void *cuda_stream);
 
 /* Synchronise the stream, read and clear the workspace's sticky device error
  * word.  *flags_out (may be NULL) receives FFD_DEVICE_FLAG_* bits.  Returns

@@ -251,7 +251,8 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
                          const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
                          void *workspace, size_t workspace_bytes, void *cuda_stream, bool requant,
                          int32_t reference, bool partials_only = false, const void *k_new = nullptr,
-                         const void *v_new = nullptr, uint64_t wait_limit_ns = kWaitLimitNs) {
+                         const void *v_new = nullptr, uint64_t wait_limit_ns = kWaitLimitNs,
+                         bool clear_counters = false) {
   ffd_status st = check_shape(s);
   if (st != FFD_OK) return st;
   if (reference != FFD_REFERENCE_RUNNING_MAX && reference != FFD_REFERENCE_SINK_LOCAL &&
@@ -333,6 +334,15 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
                   static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
   const size_t smem = decode_smem_bytes(s->block_size, group, s->split_blocks, kb.format);
+  if (clear_counters) {
+    // a shared scratch area (decode_shared_scratch): the error word and the
+    // arrival counters, which lie before the split bits, start at zero; only
+    // now that the launch is certain
+    if (L.err + 4 > L.split_bits || L.counters + static_cast<size_t>(s->batch) * s->num_kv_heads * 4 > L.split_bits)
+      return FFD_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, L.split_bits, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+      return FFD_ERR_CUDA;
+  }
   if (launch_decode(p, tmap_k, tmap_v, s->block_size, group, kb.format, grid, smem,
                     static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
     return FFD_ERR_CUDA;
@@ -356,6 +366,21 @@ uint64_t wait_limit(const ffd_decode_options *opt) {
 }
 
 }  // namespace
+
+}  // extern "C"
+
+namespace ffd {
+ffd_status decode_shared_scratch(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
+                                 const void *v_bf16, const void *k_packed, const void *k_scales,
+                                 const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                                 void *scratch, size_t scratch_bytes, void *cuda_stream) {
+  return decode_common(s, q_bf16, int4_keys(k_bf16, k_packed, k_scales), v_bf16, d_lengths, delta, out_bf16,
+                       mask, scratch, scratch_bytes, cuda_stream, false, FFD_REFERENCE_RUNNING_MAX, false,
+                       nullptr, nullptr, kWaitLimitNs, true);
+}
+}  // namespace ffd
+
+extern "C" {
 
 ffd_status ffd_decode(const ffd_shape *s, const void *q_bf16, const void *k_bf16, const void *v_bf16,
                       const void *k_packed, const void *k_scales, const int32_t *d_lengths, float delta,

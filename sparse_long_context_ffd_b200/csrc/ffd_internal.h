@@ -116,4 +116,16 @@ cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k,
                           const CUtensorMap &tmap_v, int block_size, int group, int format,
                           dim3 grid, size_t smem_bytes, cudaStream_t stream);
 
+// ffd_decode on a scratch area shared between calls (the library's own
+// device array of no_alloc.cu): every host check of ffd_decode runs first,
+// then the error word and the arrival counters are cleared on the stream,
+// then the kernel is launched.  Declared here with C++ linkage; the status
+// type comes from ffd.h.
+}  // namespace ffd
+#include "ffd.h"
+namespace ffd {
+ffd_status decode_shared_scratch(const ffd_shape *s, const void *q_bf16, const void *k_bf16,
+                                 const void *v_bf16, const void *k_packed, const void *k_scales,
+                                 const int32_t *d_lengths, float delta, void *out_bf16, uint32_t *mask,
+                                 void *scratch, size_t scratch_bytes, void *cuda_stream);
 }  // namespace ffd

@@ -12,9 +12,11 @@
 // The array costs kNoAllocScratchBytes (16 MiB) on every GPU that loads the
 // library, for the life of the process.  All calls on a device share it and
 // it keeps whatever the previous call left; the counters and the error word
-// are cleared on the stream at the start of every call.  Calls whose
-// executions overlap on the GPU (different streams, or different host
-// threads without ordering) race on the array and give undefined results.
+// are cleared on the stream at the start of every call that passes its host
+// checks.  Calls whose executions overlap on the GPU (different streams, or
+// different host threads without ordering) race on the array and give
+// undefined results.  ffd_no_alloc_device_status reads the error word that the
+// last call left (a bad length, or a bounded wait that ran out).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -35,17 +37,25 @@ std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_decode_scratch on the current device.  In host code the
-// symbol is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
-void *scratch_for_current_device() {
+// symbol is only a host-side stand-in, so the address is looked up with the
+// device current: on every call made outside a stream capture (a device reset
+// reloads this library's image, and the array may then sit elsewhere), and
+// from the copy cached by the last such call while `stream` is being captured
+// (a lookup may load the module, which a capture does not allow).
+void *scratch_for_current_device(cudaStream_t stream) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const bool capturing =
+      cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (!capturing) {
     void *ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || ptr == nullptr)
       return nullptr;
     g_scratch_ptr[dev] = ptr;
+  } else {
+    (void)cudaGetLastError();  // (a failed capture query leaves no sticky error)
   }
   return g_scratch_ptr[dev];
 }
@@ -65,14 +75,21 @@ extern "C" ffd_status ffd_decode_no_alloc(const ffd_shape *s, const void *q_bf16
   if (s->batch == 0)
     return ffd_decode(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16,
                       mask, nullptr, need, cuda_stream);
-  void *scratch = ffd::scratch_for_current_device();
+  void *scratch = ffd::scratch_for_current_device(static_cast<cudaStream_t>(cuda_stream));
   if (scratch == nullptr) return FFD_ERR_CUDA;
-  // error word and arrival counters must start at zero
-  const ffd::WorkspaceLayout L = ffd::workspace_layout(
-      s->batch, s->num_kv_heads, s->num_q_heads / s->num_kv_heads, s->capacity, s->block_size,
-      s->split_blocks);
-  if (cudaMemsetAsync(scratch, 0, L.split_bits, static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
-    return FFD_ERR_CUDA;
-  return ffd_decode(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta, out_bf16, mask,
-                    scratch, need, cuda_stream);
+  // every host check first; the array's error word and counters are cleared
+  // on the stream only once the launch is certain, so a rejected call leaves
+  // the array (and any call still running on it) alone
+  return ffd::decode_shared_scratch(s, q_bf16, k_bf16, v_bf16, k_packed, k_scales, d_lengths, delta,
+                                    out_bf16, mask, scratch, need, cuda_stream);
+}
+
+extern "C" ffd_status ffd_no_alloc_device_status(uint32_t *flags_out, void *cuda_stream) {
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+    return FFD_ERR_INVALID_ARG;  // it synchronises the stream
+  void *scratch = ffd::scratch_for_current_device(stream);
+  if (scratch == nullptr) return FFD_ERR_CUDA;
+  return ffd_check_device_status(scratch, flags_out, cuda_stream);
 }

@@ -37,7 +37,7 @@ EXPORTED = (
     "ffd_thumb_bytes", "ffd_residual_bytes", "ffd_quantize_keys_tr", "ffd_decode_tr",
     "ffd_decode_partials_tr", "ffd_decode_append", "ffd_decode_append_tr",
     "ffd_step_graph_create", "ffd_step_graph_run", "ffd_step_graph_destroy",
-    "ffd_read_probe",
+    "ffd_read_probe", "ffd_no_alloc_device_status",
 )
 
 FFD_REFERENCE_RUNNING_MAX = 0
@@ -160,6 +160,8 @@ def load_library() -> ctypes.CDLL:
             lib.ffd_decode_step.restype = st
             lib.ffd_decode_no_alloc.argtypes = [sp, p, p, p, p, p, p, ctypes.c_float, p, p, p]
             lib.ffd_decode_no_alloc.restype = st
+            lib.ffd_no_alloc_device_status.argtypes = [p, p]
+            lib.ffd_no_alloc_device_status.restype = st
             lib.ffd_check_device_status.argtypes = [p, ctypes.POINTER(ctypes.c_uint32), p]
             lib.ffd_check_device_status.restype = st
             lib.ffd_read_probe.argtypes = [p, sz, p, p]
@@ -371,11 +373,22 @@ def decode_no_alloc(shape: Shape, q, k, v, k_packed, k_scales, lengths, delta: f
     """ffd_decode without a workspace: for callers that cannot allocate device
     memory.  Uses the library's built-in 16 MiB scratch array; calls on one
     device must not overlap on the GPU.  The first call on a device should
-    come before any stream capture."""
+    come before any stream capture.  Device-side flags: no_alloc_device_status."""
     _check(load_library().ffd_decode_no_alloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
                                               _ptr(k_packed), _ptr(k_scales), _ptr(lengths),
                                               float(delta), _ptr(out), _ptr(mask),
                                               _stream(stream)), "ffd_decode_no_alloc")
+
+
+def no_alloc_device_status(stream=None) -> int:
+    """Synchronise, read and clear the flags the last decode_no_alloc call on
+    the current device left in the library's built-in array; returns
+    FFD_DEVICE_FLAG_* bits."""
+    flags = ctypes.c_uint32(0)
+    st = load_library().ffd_no_alloc_device_status(ctypes.byref(flags), _stream(stream))
+    if st not in (FFD_OK, FFD_ERR_DEVICE_CHECK, FFD_ERR_TIMEOUT):
+        raise FFDError(st, "ffd_no_alloc_device_status")
+    return int(flags.value)
 
 
 def read_probe(buf, sink, stream=None) -> None:
