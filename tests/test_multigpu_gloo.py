@@ -162,6 +162,31 @@ def test_two_rank_context_sharding_reproduces_unsharded_attention():
     assert out[0] < 1e-9 and out[1] < 1e-9
 
 
+def _gather_worker(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    from sparse_long_context_ffd_b200 import sharded
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    bench.dist_init("gloo", world)
+    try:
+        region = torch.arange(37, dtype=torch.int64).to(torch.uint8) + 100 * rank
+        got = sharded.gather_regions(region)
+        out[rank] = got.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_regions_concatenates_in_rank_order_over_gloo():
+    # the exchange step of the context-sharded decode (sharded.sharded_decode)
+    world = 2
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_gather_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    want = np.concatenate([np.arange(37, dtype=np.uint8) + 100 * r for r in range(world)])
+    assert np.array_equal(out[0], want) and np.array_equal(out[1], want)
+
+
 def test_shard_bookkeeping():
     from sparse_long_context_ffd_b200 import sharded
     ll = [sharded.local_lengths([0, 100, 256, 700], r, 256) for r in range(3)]
