@@ -583,15 +583,17 @@ def oracle_step_sample(w, inp, budget_s: float):
     key = (w.name, w.seed)
     if key not in _ORACLE_RATE:
         n = min(n0, split_tok)
-        p, s = oracle.quantize_keys(inp["k"][:1, :1, :n], np.array([n], np.int32), T)
+        c = -(-n // T) * T  # cache rows of the sample: whole blocks
+        p, s = oracle.quantize_keys(inp["k"][:1, :1, :c], np.array([n], np.int32), T)
         t0 = time.perf_counter()
-        oracle.decode(inp["q"][:1, :G], inp["k"][:1, :1, :n], inp["v"][:1, :1, :n], p, s,
+        oracle.decode(inp["q"][:1, :G], inp["k"][:1, :1, :c], inp["v"][:1, :1, :c], p, s,
                       np.array([n], np.int32), T, S, w.delta)
         _ORACLE_RATE[key] = max((time.perf_counter() - t0) / n, 1e-9)
     rate = _ORACLE_RATE[key]
     n = int(budget_s / rate) // split_tok * split_tok
     n = max(min(n0, split_tok), min(n0, n))
-    k1, v1 = inp["k"][:1, :1, :n], inp["v"][:1, :1, :n]
+    c = -(-n // T) * T
+    k1, v1 = inp["k"][:1, :1, :c], inp["v"][:1, :1, :c]
     p1, s1 = oracle.quantize_keys(k1, np.array([n], np.int32), T)
     ln = np.array([n], np.int32)
     reps, tokens = 0, 0
@@ -657,38 +659,54 @@ def host_cpu() -> dict:
 
 
 def oracle_parallel_sample(w, inp, budget_s: float):
-    """The oracle as it stands, on several host cores at once: one process per
-    kv-head group of sequence 0 (independent units of the step), each over the
-    same prefix of whole splits as the single-thread sample, all started
-    together; scaled by token count to the full step.  Returns (us per full
+    """The oracle as it stands, on every host core at once: one process per
+    core, each running one decode step (last-block re-quantisation + the whole
+    oracle step) of one kv-head group over a window of whole splits.  Jobs go
+    round-robin over all (sequence, kv-head) units of the step, and each job's
+    window starts at a different split of its sequence, so the sample covers
+    the whole workload; splits are independent units of the method, so a
+    window is a fair share of the step.  All start together; the slowest sets
+    the time, scaled by token count to the full step.  Returns (us per full
     step, cores, description)."""
     import concurrent.futures
     import multiprocessing
     T, S, G = w.block_size, w.split_blocks, w.group
-    units = w.num_kv_heads
-    cores = max(1, min(os.cpu_count() or 1, units, 16))
-    n0 = int(inp["lengths"][0])
+    cores = max(1, os.cpu_count() or 1)
     split_tok = S * T
     rate = _ORACLE_RATE.get((w.name, w.seed))
     if rate is None:
         oracle_step_sample(w, inp, min(budget_s, 2.0))
         rate = _ORACLE_RATE[(w.name, w.seed)]
-    n = int(budget_s / rate) // split_tok * split_tok
-    n = max(min(n0, split_tok), min(n0, n))
-    jobs = [(np.ascontiguousarray(inp["q"][:1, g * G:(g + 1) * G]),
-             np.ascontiguousarray(inp["k"][:1, g:g + 1, :n]),
-             np.ascontiguousarray(inp["v"][:1, g:g + 1, :n]), n, T, S, w.delta, 1)
-            for g in range(cores)]
+    lengths = inp["lengths"]
+    units = [(b, g) for b in range(w.batch) for g in range(w.num_kv_heads) if int(lengths[b]) > 0]
+    n = max(split_tok, int(budget_s / rate) // split_tok * split_tok)
+    jobs = []
+    for c in range(cores):
+        b, g = units[c % len(units)]
+        nb_tok = int(lengths[b])
+        win = min(n, nb_tok)
+        nsplits = max(1, -(-nb_tok // split_tok))
+        t0 = ((c // len(units)) * 7 + c) % nsplits * split_tok  # a different split per job
+        t0 = min(t0, max(0, nb_tok - win)) // split_tok * split_tok
+        win = min(win, nb_tok - t0)
+        cap_j = -(-win // T) * T  # the window's cache rows: whole blocks
+        jobs.append((np.ascontiguousarray(inp["q"][b:b + 1, g * G:(g + 1) * G]),
+                     np.ascontiguousarray(inp["k"][b:b + 1, g:g + 1, t0:t0 + cap_j]),
+                     np.ascontiguousarray(inp["v"][b:b + 1, g:g + 1, t0:t0 + cap_j]), win, T, S,
+                     w.delta, 1))
     ctx = multiprocessing.get_context("spawn")  # the parent has a CUDA context
     with concurrent.futures.ProcessPoolExecutor(max_workers=cores, mp_context=ctx) as ex:
         list(ex.map(_oracle_unit_worker, [j[:7] + (0,) for j in jobs]))  # start and load the workers
         elapsed = list(ex.map(_oracle_unit_worker, jobs))
     wall = max(elapsed)
-    full_tokens = int(np.sum(inp["lengths"])) * w.num_kv_heads
-    us = wall / (cores * n) * full_tokens * 1e6
-    desc = (f"{cores} host processes at once, each one kv-head group (G={G}) of sequence 0 over "
-            f"its first {n} tokens (one step each); scaled by token count to the full step "
-            f"({full_tokens} token-heads)")
+    tokens = sum(j[3] for j in jobs)
+    full_tokens = int(np.sum(lengths)) * w.num_kv_heads
+    us = wall / tokens * full_tokens * 1e6
+    desc = (f"{cores} host processes at once (every core), job c = one decode step of kv-head "
+            f"group (b, g) = unit c mod {len(units)} (all (sequence, kv-head) units of the step) "
+            f"over a window of whole splits ({n} tokens, at most the sequence) starting at a "
+            f"different split per job; {tokens} token-heads in all, scaled by token count to the "
+            f"full step ({full_tokens} token-heads)")
     return us, cores, desc
 
 

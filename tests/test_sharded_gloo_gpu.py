@@ -70,7 +70,7 @@ def _rank(rank, world, port, cfg, out):
                          ids=["T64S4G4", "T64S2G8", "T128S3G2dense"])
 def test_two_gloo_ranks_exchange_the_library_region(cfg):
     world = 2
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()  # (this process already holds a CUDA context)
     out = manager.dict()
     mp.spawn(_rank, args=(world, _free_port(), cfg, out), nprocs=world, join=True)
     T, S, G, Hkv, B, delta, seed = cfg
