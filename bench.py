@@ -950,6 +950,16 @@ def run_gpu(args):
     if not args.no_tr:
         tr = measure_thumb_resid(w, inp, device, args, world, l2)
 
+    # the method's own regime beside the headline: the same shape with
+    # concentrated attention, where few blocks are kept (timing only; the
+    # oracle checks these rows in --rho-sweep and in the GPU tests)
+    rho = None
+    if not args.no_rho:
+        rho = [rho_row(name, ref_name, REFERENCES[ref_name], device, min(args.steps, 200),
+                       min(args.warmup, 10), world, load_peaks()[0], l2, check=False)
+               for name, ref_name in (("rho1of64", "running"), ("rho0p05", "running"),
+                                      ("rho1of64", "sink_local_fixed"))]
+
     e2e = None
     if not args.no_e2e:
         del rep
@@ -1011,6 +1021,10 @@ def run_gpu(args):
                            "achieved_gbs": (algo_dense["total"] / (dense_decode_ms * 1e-3) / 1e9)
                            if dense_decode_ms else None},
             "thumb_residual": tr,
+            "kept_fraction_sweep": ({"workload": "long-context shape (B1 Hq32 Hkv8 N131072 T64 S64 "
+                                                 "delta 3) with concentrated attention "
+                                                 "(ffd_workloads.RHO_DOMINANT)",
+                                     "rows": rho} if rho else None),
             "e2e": ({"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                      "d2h_bytes_per_step": e2e["d2h"],
                      "wall_ms_per_step": e2e["wall_ms_per_step"],
@@ -1088,6 +1102,54 @@ def run_context_sweep(args):
     return 0
 
 
+def rho_row(name, ref_name, ref, device, steps, warmup, world, peak, l2, check=True, inp=None,
+            dense=False):
+    """One row of the kept-fraction sweep: the fused step on a controlled-
+    sparsity workload (ffd_workloads.RHO_DOMINANT) with one reference maximum,
+    timed from CUDA graphs; optionally checked against the oracle (mask
+    bit-exact, output max-abs / mean-abs) on the same inputs."""
+    import torch
+    w = fw.WORKLOADS[name]
+    if inp is None:
+        inp = fw.make_inputs(w)
+    probe = Replica(w, inp, device, 1)
+    probe.reference = ref
+    probe.step(0, w.delta)
+    torch.cuda.synchronize(device)
+    mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
+    out = probe.layers[0]["bufs"].out.float().cpu().numpy().astype(np.float64)
+    kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
+    algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)["total"]
+    del probe
+    row = {"workload": name, "reference": ref_name,
+           "kept_fraction": kept_blocks / max(1, valid_blocks), "algorithmic_bytes": algo}
+    if check:
+        import oracle
+        packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+        sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+        _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
+                                     w.split_blocks, w.delta, reference=ref)
+        want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
+                                    w.block_size)
+        err = np.abs(out - want_out)
+        row["oracle"] = {"mask_equal": bool(np.array_equal(mask, want_mask)),
+                         "max_abs": float(err.max()), "mean_abs": float(err.mean())}
+    layers = max(1, min(64, math.ceil(3 * l2 / algo)))
+    rep = Replica(w, inp, device, layers)
+    rep.reference = ref
+    _, per, _ = time_graph_steps(rep, w.delta, steps, warmup, world, device)
+    us = dist_max(float(np.mean(per)) * 1e3, world, device)
+    row.update({"decode_us": us, "tbs": algo / (us * 1e-6) / 1e12,
+                "frac": algo / (us * 1e-6) / 1e9 / peak})
+    if dense:
+        _, per_d, _ = time_graph_steps(rep, float("inf"), steps, warmup, world, device)
+        row["dense_us"] = dist_max(float(np.mean(per_d)) * 1e3, world, device)
+    rep.check_flags()
+    del rep
+    torch.cuda.empty_cache()
+    return row
+
+
 def run_rho_sweep(args):
     """The method's own regime: decode time against the kept fraction.  The
     long-context shape with concentrated attention (ffd_workloads.RHO_DOMINANT:
@@ -1097,54 +1159,23 @@ def run_rho_sweep(args):
     kernel in dense mode.  Each row is checked against the oracle on the same
     inputs (mask bit-exact, output max-abs / mean-abs), one JSON line."""
     import torch
-    import oracle
-    from sparse_long_context_ffd_b200 import ffd
     device = torch.device("cuda", torch.cuda.current_device())
     l2 = getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 126 * 2**20)
     peak, peak_src = load_peaks()
-    refs = [("running", ffd.FFD_REFERENCE_RUNNING_MAX), ("sink_local_fixed", ffd.FFD_REFERENCE_SINK_LOCAL_FIXED)]
+    refs = [("running", REFERENCES["running"]), ("sink_local_fixed", REFERENCES["sink_local_fixed"])]
     rows = []
     dense_us = None
+    steps = min(args.steps, 400)
     for name in fw.RHO_DOMINANT:
-        w = fw.WORKLOADS[name]
-        inp = fw.make_inputs(w)
-        packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
-        sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+        inp = fw.make_inputs(fw.WORKLOADS[name])
         for ref_name, ref in refs:
-            probe = Replica(w, inp, device, 1)
-            probe.reference = ref
-            probe.step(0, w.delta)
-            torch.cuda.synchronize(device)
-            mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
-            out = probe.layers[0]["bufs"].out.float().cpu().numpy().astype(np.float64)
-            kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
-            _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
-                                         w.split_blocks, w.delta, reference=ref)
-            want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
-                                        w.block_size)
-            err = np.abs(out - want_out)
-            algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)["total"]
-            del probe
-            layers = max(1, min(64, math.ceil(3 * l2 / algo)))
-            rep = Replica(w, inp, device, layers)
-            rep.reference = ref
-            _, per, _ = time_graph_steps(rep, w.delta, min(args.steps, 400), args.warmup, 1, device)
-            if dense_us is None:
-                _, per_d, _ = time_graph_steps(rep, float("inf"), min(args.steps, 400), args.warmup, 1,
-                                               device)
-                dense_us = float(np.mean(per_d)) * 1e3
-            rep.check_flags()
-            us = float(np.mean(per)) * 1e3
-            rows.append({"workload": name, "reference": ref_name,
-                         "kept_fraction": kept_blocks / max(1, valid_blocks),
-                         "decode_us": us, "algorithmic_bytes": algo,
-                         "tbs": algo / (us * 1e-6) / 1e12, "frac": algo / (us * 1e-6) / 1e9 / peak,
-                         "dense_us": dense_us, "vs_dense": dense_us / us,
-                         "oracle": {"mask_equal": bool(np.array_equal(mask, want_mask)),
-                                    "max_abs": float(err.max()), "mean_abs": float(err.mean())}})
-            del rep
-            torch.cuda.empty_cache()
-        del inp, packed, scales, sc
+            row = rho_row(name, ref_name, ref, device, steps, args.warmup, 1, peak, l2, check=True,
+                          inp=inp, dense=dense_us is None)
+            dense_us = row.get("dense_us", dense_us)
+            row["dense_us"] = dense_us
+            row["vs_dense"] = dense_us / row["decode_us"]
+            rows.append(row)
+        del inp
     line = {"mode": "rho-sweep", "metric": "us per decode launch vs kept fraction (128K)",
             "unit": "us",
             "workload": "long-context shape (B1 Hq32 Hkv8 D128 N131072 T64 S64 delta 3) with "
@@ -1174,6 +1205,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rho", action="store_true",
+                    help="skip the small-kept-fraction rows of the default line")
     ap.add_argument("--no-tr", action="store_true",
                     help="skip the thumbnail + residual format measurement")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

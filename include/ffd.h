@@ -99,8 +99,12 @@ size_t ffd_mask_words(const ffd_shape *shape);
 
 /* Device workspace ffd_decode needs: split partials (running max, sum and
  * unnormalised output per head), per-split selection bits, one arrival
- * counter per (b, kv-head) and the sticky device error word.  0 for an
- * invalid shape. */
+ * counter per (b, kv-head) and the sticky device error word.  When the
+ * splits alone would leave SMs idle, R CTAs share each split (R the largest
+ * power of two up to 8 and up to S with B * Hkv * ceil(nblk / S) * R <= 296,
+ * two CTAs on each of a B200's 148 SMs): each scans the whole split, so all
+ * take the same selection with no exchange, and attends over every R-th kept
+ * block; the partials then hold R slots per split.  0 for an invalid shape. */
 size_t ffd_decode_workspace_bytes(const ffd_shape *shape);
 
 /* Zero a workspace (cudaMemsetAsync on the stream).  Call once after

@@ -90,12 +90,23 @@ bool make_resid_tensor_map(CUtensorMap *map, const void *base, uint64_t rows) {
 
 }  // namespace
 
+int32_t parts_per_split(int32_t batch, int32_t num_kv_heads, int32_t capacity, int32_t block_size,
+                        int32_t split_blocks) {
+  constexpr int64_t kSlots = 2 * 148;  // two CTAs per SM on a B200
+  const int64_t nblk = capacity / block_size;
+  const int64_t units = static_cast<int64_t>(batch) * num_kv_heads * ((nblk + split_blocks - 1) / split_blocks);
+  int32_t r = 1;
+  while (r < 8 && 2 * r <= split_blocks && units * 2 * r <= kSlots) r *= 2;
+  return r;
+}
+
 WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group, int32_t capacity,
-                                 int32_t block_size, int32_t split_blocks) {
+                                 int32_t block_size, int32_t split_blocks, int32_t parts) {
   WorkspaceLayout L{};
   const int64_t nblk = capacity / block_size;
   L.nsplit_max = static_cast<int32_t>((nblk + split_blocks - 1) / split_blocks);
   L.split_words = (split_blocks + 31) / 32;
+  L.parts = parts;
   const size_t rows = static_cast<size_t>(batch) * num_kv_heads;
   size_t off = 0;
   L.err = off;
@@ -105,7 +116,7 @@ WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t gr
   L.split_bits = off;
   off += round_up(rows * L.nsplit_max * L.split_words * 4, 256);
   L.partials = off;
-  off += rows * L.nsplit_max * group * kPartialStride * 4;
+  off += rows * L.nsplit_max * parts * group * kPartialStride * 4;
   L.total = round_up(off, 256);
   return L;
 }
@@ -160,7 +171,8 @@ size_t ffd_mask_words(const ffd_shape *s) {
 size_t ffd_decode_workspace_bytes(const ffd_shape *s) {
   if (check_shape(s) != FFD_OK) return 0;
   return workspace_layout(s->batch, s->num_kv_heads, s->num_q_heads / s->num_kv_heads, s->capacity,
-                          s->block_size, s->split_blocks)
+                          s->block_size, s->split_blocks,
+                          parts_per_split(s->batch, s->num_kv_heads, s->capacity, s->block_size, s->split_blocks))
       .total;
 }
 
@@ -269,8 +281,12 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   const bool dense = std::isinf(delta);
   const bool tr = kb.format == kFormatThumbResid;
   const int group = s->num_q_heads / s->num_kv_heads;
+  // a context shard keeps one CTA per split: its exchanged region is the
+  // one-part layout that ffd_partials_region names
+  const int32_t parts = partials_only ? 1 : parts_per_split(s->batch, s->num_kv_heads, s->capacity,
+                                                            s->block_size, s->split_blocks);
   const WorkspaceLayout L =
-      workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks);
+      workspace_layout(s->batch, s->num_kv_heads, group, s->capacity, s->block_size, s->split_blocks, parts);
   if (workspace == nullptr || workspace_bytes < L.total) return FFD_ERR_WORKSPACE;
   if (q_bf16 == nullptr || v_bf16 == nullptr || d_lengths == nullptr ||
       (!partials_only && (out_bf16 == nullptr || mask == nullptr)))
@@ -321,6 +337,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   p.requant_last = requant ? 1 : 0;
   p.reference = reference;
   p.partials_only = partials_only ? 1 : 0;
+  p.parts = L.parts;
   p.wait_limit_ns = wait_limit_ns;
   p.k = static_cast<const uint16_t *>(kb.k);
   p.packed_out = requant ? static_cast<uint8_t *>(const_cast<void *>(kb.packed)) : nullptr;
@@ -331,7 +348,7 @@ ffd_status decode_common(const ffd_shape *s, const void *q_bf16, const KeyBuffer
   p.k_out = append ? static_cast<uint16_t *>(const_cast<void *>(kb.k)) : nullptr;
   p.v_out = append ? static_cast<uint16_t *>(const_cast<void *>(v_bf16)) : nullptr;
 
-  const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max : 1),
+  const dim3 grid(static_cast<unsigned>(L.nsplit_max > 0 ? L.nsplit_max * L.parts : 1),
                   static_cast<unsigned>(s->num_kv_heads), static_cast<unsigned>(s->batch));
   const size_t smem = decode_smem_bytes(s->block_size, group, s->split_blocks, kb.format);
   if (clear_counters) {

@@ -68,6 +68,10 @@ constexpr int kKvHalfBytes = kKvTok * 128;          // one 64-channel half of K 
 constexpr int kMergeBytes = kAttnWarps * (8 + 8 + 8 * kHeadDim) * 4;
 // block quantiser scratch for the attention warps: per-warp channel maxima + scales
 constexpr int kRequantScratchBytes = (kAttnWarps + 1) * kHeadDim * 4;
+// Scored scan entries waiting for the in-order Top-delta decision: entry e
+// uses slot e % kScanSlots, so at most kScanSlots entries are claimed ahead of
+// the decision frontier.
+constexpr int kScanSlots = 16;
 
 // One attention stage (kKvTok tokens of one kept block) per key format.
 template <int F>
@@ -94,7 +98,9 @@ template <int T, int F>
 struct ScanGeom {
   static constexpr int kRowBytes = F == kFormatThumbResid ? kThumbRowBytes : kPackedRowBytes;
   static constexpr int kStageBytes = T * kRowBytes + kScaleRowBytes;
-  static constexpr int kStages = (F == kFormatThumbResid ? 2 : 1) * (T == 64 ? 4 : 2);
+  // As many stages as fit beside the K/V ring with two CTAs per SM: several
+  // warps score entries at once, and each holds its stage while it reads it.
+  static constexpr int kStages = F == kFormatThumbResid ? (T == 64 ? 9 : 5) : (T == 64 ? 6 : 3);
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
 };
@@ -108,10 +114,16 @@ struct SmemLayout {
   static constexpr int kNumBars = 2 * ScanGeom<T, F>::kStages + 2 * NKV;
   static constexpr int kMeta = kBars + 8 * kNumBars;  // int [NKV] token offsets
   static constexpr int kSeq = kMeta + 4 * NKV;        // int [NKV] item indices
-  static constexpr int kCtrl = kSeq + 4 * NKV;        // qcount, sel_done, is_last, abort, requant_done
-  static constexpr int kRequant = kCtrl + 32;         // re-quantisation scratch (attention warps)
+  // qcount, sel_done, is_last, abort, requant_done, scan claim, scan decided
+  static constexpr int kCtrl = (kSeq + 4 * NKV + 15) / 16 * 16;
+  static constexpr int kScanSeq = kCtrl + 32;                // int [NSA] scan entry per stage
+  static constexpr int kSlotSeq = kScanSeq + 4 * kScanSlots;  // int [kScanSlots] entry per slot
+  static constexpr int kScores = kSlotSeq + 4 * kScanSlots;   // float [kScanSlots][8]
+  static constexpr int kQRows = kScores + 32 * kScanSlots;    // bf16 [8][128]: the query group
+  static constexpr int kRequant = kQRows + 8 * kHeadDim * 2;  // re-quantisation scratch (attention warps)
   static constexpr int kKeep = kRequant + kRequantScratchBytes;  // u32 [split_words]
   // queue of kept block indices (u16 [split_blocks]) follows keep bits
+  static_assert(ScanGeom<T, F>::kStages <= kScanSlots, "one sequence word per scan stage");
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -242,14 +254,11 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t 
 // to +-127 never acts.  When 127 / a overflows (a below about 3.7e-37), or a
 // itself is infinite, the conversion is done the direct way instead.
 template <int G, int F>
-__device__ __forceinline__ void fold_block(const uint16_t *scl, const uint32_t (&qv)[ScanFold<G, F>::NC / 2],
-                                           int lane, uint32_t (&bq)[8], int &sumq, float &a_out) {
+__device__ __forceinline__ void fold_block_sv(const uint32_t (&sv)[ScanFold<G, F>::NC / 2],
+                                              const uint32_t (&qv)[ScanFold<G, F>::NC / 2], int lane,
+                                              uint32_t (&bq)[8], int &sumq, float &a_out) {
   using SF = ScanFold<G, F>;
   constexpr int NC = SF::NC, NW = SF::NW, R = SF::R;
-  const int gid = lane >> 2, t4 = lane & 3;
-  const int r = SF::part(gid);
-  uint32_t sv[NC / 2];
-  SF::load_pairs(scl + 32 * t4, r, sv);
   // p_c is recomputed where it is used (an exact product) rather than kept
   auto pc = [&](int c) {
     return (c & 1) ? __fmul_rn(bf16_hi(qv[c >> 1]), bf16_hi(sv[c >> 1])) : __fmul_rn(bf16_lo(qv[c >> 1]), bf16_lo(sv[c >> 1]));
@@ -313,6 +322,16 @@ __device__ __forceinline__ void fold_block(const uint16_t *scl, const uint32_t (
   }
   sumq = sq;
   a_out = a;
+}
+
+// fold_block_sv with the lane's scale pairs read from a block's scale row.
+template <int G, int F>
+__device__ __forceinline__ void fold_block(const uint16_t *scl, const uint32_t (&qv)[ScanFold<G, F>::NC / 2],
+                                           int lane, uint32_t (&bq)[8], int &sumq, float &a_out) {
+  using SF = ScanFold<G, F>;
+  uint32_t sv[SF::NC / 2];
+  SF::load_pairs(scl + 32 * (lane & 3), SF::part(lane >> 2), sv);
+  fold_block_sv<G, F>(sv, qv, lane, bq, sumq, a_out);
 }
 
 // Selector, tensor-core part: the integer score sum_c qi_c u_c of every token
@@ -398,6 +417,106 @@ __device__ __forceinline__ void block_scores(int best0, int best1, int sumq, flo
   }
 }
 
+// ------------------------------------------------------------------------
+// Cooperative selector.  Scoring a block (fold + integer scan + block score)
+// is independent from block to block; only the Top-delta decision runs in
+// block order (the running maximum).  So the scan warp and, while they wait
+// for K/V, the attention warps all score scan entries: a warp claims the next
+// entry (ctrl[5], in order), scores it from its ring stage, releases the
+// stage and leaves the head scores in slot e % kScanSlots with e written
+// last into the slot's sequence word.  The scan warp alone decides, entry by
+// entry in order, from the slots (ctrl[6] counts the decided entries and
+// frees their slots).  Max is taken in the same order as a single scanning
+// warp would, so the selection is bit-identical to it.
+
+struct ScanShared {
+  volatile int *ctrl;       // [5] next entry to claim, [6] entries decided
+  volatile int *scan_seq;   // [stage]: entry whose tile the producer put there
+  volatile int *slot_seq;   // [slot]: entry whose scores the slot holds
+  float *scores;            // [slot][8 heads]
+  const uint16_t *q_rows;   // [G][128]: the query group
+};
+
+// Lane 0 claims the next scan entry; the whole warp gets the result: the
+// entry, -1 once every entry is claimed, -2 if none can be taken now (the
+// slot window is full, or -- when `landed_only` -- its tile has not landed).
+template <int NSA>
+__device__ __forceinline__ int claim_scan_entry(const ScanShared &sh, uint64_t *full_a, int total, bool landed_only,
+                                                int lane) {
+  int e = -2;
+  if (lane == 0) {
+    const int c = sh.ctrl[5];
+    if (c >= total) {
+      e = -1;
+    } else if (c < sh.ctrl[6] + kScanSlots) {
+      const int st = c % NSA;
+      const bool ready = !landed_only ||
+                         (sh.scan_seq[st] == c && mbar_test_wait(&full_a[st], static_cast<uint32_t>(c / NSA) & 1u));
+      if (ready && atomicCAS(const_cast<int *>(&sh.ctrl[5]), c, c + 1) == c) e = c;
+    }
+  }
+  return __shfl_sync(kFull, e, 0);
+}
+
+// Score scan entry e (block jb, valid_rows tokens): wait for its tile (the
+// producer's sequence word, then the stage's fill, both bounded), fold the
+// query with the block's scales, scan, release the stage.  s0, s1: the
+// scores of heads 2 t4 and 2 t4 + 1 (every lane).  False if a wait ran out.
+template <int T, int G, int F>
+__device__ __forceinline__ bool score_scan_entry(const ScanShared &sh, uint8_t *scan_ring, uint64_t *full_a,
+                                                 uint64_t *empty_a, int e, int valid_rows, int lane,
+                                                 uint64_t limit_ns, float &s0, float &s1) {
+  using SG = ScanGeom<T, F>;
+  using SF = ScanFold<G, F>;
+  constexpr int NSA = SG::kStages;
+  const int st = e % NSA;
+  if (!wait_item_published(sh.scan_seq, st, e, limit_ns) ||
+      !mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, limit_ns))
+    return false;
+  const int gid = lane >> 2, t4 = lane & 3;
+  const uint8_t *tile = scan_ring + st * SG::kStageBytes;
+  uint32_t qv[SF::NC / 2];
+  SF::load_pairs(sh.q_rows + (gid % G) * kHeadDim + 32 * t4, SF::part(gid), qv);
+  uint32_t bq[8];
+  int sq, best0, best1;
+  float am;
+  fold_block<G, F>(reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes), qv, lane, bq, sq, am);
+  block_best<T, F>(tile, bq, valid_rows, lane, best0, best1);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&empty_a[st]);
+  block_scores<F>(best0, best1, sq, am, lane, s0, s1);
+  return true;
+}
+
+// Leave scan entry e's head scores in its slot, e written last into the
+// slot's sequence word (for the scan warp's in-order decision).
+__device__ __forceinline__ void publish_scan_scores(const ScanShared &sh, int e, float s0, float s1, int lane) {
+  float *slot = sh.scores + (e % kScanSlots) * 8;
+  if (lane < 4) {  // lane t4 holds heads 2 t4 and 2 t4 + 1
+    slot[2 * lane] = s0;
+    slot[2 * lane + 1] = s1;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence_block();
+    sh.slot_seq[e % kScanSlots] = e;
+  }
+}
+
+// The attention warps' call: kept out of line, so that the registers it needs
+// do not raise the attention loop's own allocation (the live registers of the
+// caller are saved around the call, which happens only while it waits).
+template <int T, int G, int F>
+__device__ __noinline__ bool score_scan_entry_helper(const ScanShared &sh, uint8_t *scan_ring, uint64_t *full_a,
+                                                     uint64_t *empty_a, int e, int valid_rows, int lane,
+                                                     uint64_t limit_ns) {
+  float s0, s1;
+  if (!score_scan_entry<T, G, F>(sh, scan_ring, full_a, empty_a, e, valid_rows, lane, limit_ns, s0, s1))
+    return false;
+  publish_scan_scores(sh, e, s0, s1, lane);
+  return true;
+}
+
 template <int T, int G, int F>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -425,10 +544,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   // qcount, sel_done, is_last, abort, requant_done
   volatile int *ctrl = reinterpret_cast<volatile int *>(smem + SL::kCtrl);
   uint32_t *keepbits = reinterpret_cast<uint32_t *>(smem + SL::kKeep);
+  const ScanShared sh{ctrl, reinterpret_cast<volatile int *>(smem + SL::kScanSeq),
+                      reinterpret_cast<volatile int *>(smem + SL::kSlotSeq),
+                      reinterpret_cast<float *>(smem + SL::kScores),
+                      reinterpret_cast<const uint16_t *>(smem + SL::kQRows)};
   volatile uint16_t *queue =
       reinterpret_cast<volatile uint16_t *>(keepbits + ((p.split_words + 3) & ~3));
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  // R = p.parts CTAs per split when the splits alone leave SMs idle: every
+  // one of them scans the whole split (so all take the same decisions, with
+  // no exchange) and attends over its share of the kept blocks (kept-list
+  // positions = part mod R); each writes its own partial.
+  const int R = p.parts;
+  const int split = blockIdx.x / R, part = blockIdx.x % R, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_q_heads = p.num_kv_heads * G;
   const int len = p.lengths[b];
@@ -441,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (split >= nsplit) {
     // Empty or invalid sequence: split 0 writes zero rows and an empty mask.
-    if (split == 0) {
+    if (split == 0 && part == 0) {
       if (bad && threadIdx.x == 0 && g == 0) atomicOr(p.err, kFlagBadLength);
       if (!p.partials_only &&
           FFD_IN_BOUNDS(p, row < static_cast<size_t>(p.batch) * p.num_kv_heads)) {  // (a shard leaves them to the merge)
@@ -472,14 +600,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&empty_b[s], 1);
       seq[s] = -1;
     }
-    ctrl[0] = 0;
-    ctrl[1] = 0;
-    ctrl[2] = 0;
-    ctrl[3] = 0;
-    ctrl[4] = 0;
+    for (int c = 0; c < 7; ++c) ctrl[c] = 0;
+    for (int s = 0; s < NSA; ++s) sh.scan_seq[s] = -1;
+    for (int s = 0; s < kScanSlots; ++s) sh.slot_seq[s] = -1;
     fence_mbar_init();
   }
   for (int w = threadIdx.x; w < p.split_words; w += blockDim.x) keepbits[w] = 0u;
+  // the query group, for every warp that scores scan entries
+  for (int i = threadIdx.x; i < G * kHeadDim / 8; i += blockDim.x)
+    reinterpret_cast<uint4 *>(smem + SL::kQRows)[i] = reinterpret_cast<const uint4 *>(
+        p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim)[i];
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
@@ -531,6 +661,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (jb == nb - 1 && !requant_ready()) break;
         if (use > 0 && !mbar_test_wait(&empty_a[st], static_cast<uint32_t>(use - 1) & 1u)) break;
         uint8_t *dst = scan_ring + st * SG::kStageBytes;
+        sh.scan_seq[st] = sc_next;
         mbar_arrive_expect_tx(&full_a[st], SG::kStageBytes);
         if (FFD_IN_BOUNDS(p, jb >= 0 && (jb + 1) * T <= p.capacity && row_ok)) {
           bulk_g2s(dst, src_p + static_cast<size_t>(jb) * T * SG::kRowBytes, T * SG::kRowBytes,
@@ -546,6 +677,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool sel_done = dense || ld_acquire_cta(&ctrl[1]) != 0;
       const int avail = dense ? nbs : ld_acquire_cta(&ctrl[0]);
       while (q_ptr < avail) {
+        if (q_ptr % R != part) {  // another part's block
+          ++q_ptr;
+          continue;
+        }
         const int j = dense ? q_ptr : static_cast<int>(queue[q_ptr]);
         const int tok = (j0 + j) * T + sub * kKvTok;
         if (sub >= kSubPerBlock || tok >= len) {
@@ -617,13 +752,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ============================================================ scan warp
   if (warp == kScanWarp) {
     if (dense) return;
-    using SF = ScanFold<G, F>;
     const int gid = lane >> 2, t4 = lane & 3;
-    // the lane's query channels in its fold order (see ScanFold)
-    uint32_t qv[SF::NC / 2];
-    SF::load_pairs(p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid % G) *
-                             kHeadDim + 32 * t4,
-                   SF::part(gid), qv);
     float run0 = -INFINITY, run1 = -INFINITY;  // running max of heads 2*t4, 2*t4 + 1
     // the pages' rule: the pseudo-max is a fixed threshold (no running update)
     const bool fixed_ref = p.reference == 2;
@@ -658,24 +787,64 @@ __global__ void __launch_bounds__(kThreads, 2)
         ++qn;
       }
     };
-    for (int e = 0; e < nref + nbs; ++e) {
-      const int st = e % NSA;
-      if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, p.wait_limit_ns)) {
+    // score entries (the attention warps help while they wait for K/V) and
+    // decide them in block order
+    const int total = nref + nbs;
+    int decided = 0;
+    uint64_t idle_since = 0;
+    while (true) {
+      bool progress = false;
+      while (decided < total) {
+        const int ready = __shfl_sync(kFull, lane == 0 ? sh.slot_seq[decided % kScanSlots] == decided : 0, 0);
+        if (!ready) break;
+        __threadfence_block();
+        const float *slot = sh.scores + (decided % kScanSlots) * 8;
+        decide(decided, slot[2 * t4], slot[2 * t4 + 1]);
+        ++decided;
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          ctrl[6] = decided;  // frees the entry's slot
+        }
+        progress = true;
+      }
+      if (decided >= total || __shfl_sync(kFull, lane == 0 ? ctrl[3] : 0, 0)) break;
+      // (the next entry whether or not its tile has landed: the scan warp
+      // then waits on the stage's barrier rather than polling)
+      const int e = claim_scan_entry<NSA>(sh, full_a, total, false, lane);
+      if (e >= 0) {
+        const int jb = scan_block_index(e, nref, nb, j0);
+        float s0, s1;
+        if (!score_scan_entry<T, G, F>(sh, scan_ring, full_a, empty_a, e, min(T, len - jb * T), lane,
+                                       p.wait_limit_ns, s0, s1)) {
+          raise_timeout(p, ctrl);
+          break;
+        }
+        if (e == decided) {  // next in order: decide at once, no slot
+          decide(e, s0, s1);
+          ++decided;
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence_block();
+            ctrl[6] = decided;
+          }
+        } else {
+          publish_scan_scores(sh, e, s0, s1, lane);
+        }
+        progress = true;
+      }
+      if (progress) {
+        idle_since = 0;
+        continue;
+      }
+      const uint64_t now = global_timer_ns();
+      if (idle_since == 0) {
+        idle_since = now;
+      } else if (now - idle_since > p.wait_limit_ns) {
         raise_timeout(p, ctrl);
         break;
       }
-      const int jb = scan_block_index(e, nref, nb, j0);
-      const uint8_t *tile = scan_ring + st * SG::kStageBytes;
-      uint32_t bq[8];
-      int sq, best0, best1;
-      float am, s0, s1;
-      fold_block<G, F>(reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes), qv, lane, bq, sq, am);
-      block_best<T, F>(tile, bq, min(T, len - jb * T), lane, best0, best1);
-      block_scores<F>(best0, best1, sq, am, lane, s0, s1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_a[st]);
-      decide(e, s0, s1);
-      if (ctrl[3]) break;
+      __nanosleep(20);
     }
     if (lane == 0) {
       __threadfence_block();
@@ -765,7 +934,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                                       new_k_row);
     fence_proxy_async_smem();  // both regions are later written by async copies
     named_barrier(2, kAttnThreads);
-    if (threadIdx.x == 0) mbar_arrive(&full_a[1]);
+    if (threadIdx.x == 0) {
+      sh.scan_seq[1] = 1;
+      mbar_arrive(&full_a[1]);
+    }
   }
   float m_run[2] = {-INFINITY, -INFINITY};  // heads 2*t4, 2*t4 + 1
   float l_run[2] = {0.0f, 0.0f};
@@ -787,6 +959,36 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   for (int it = warp;; it += kAttnWarps) {
     const int st = it % NKV;
+    // Until item `it` is published, score scan entries whose tiles have
+    // landed (the selector's work, decided in order by the scan warp).  Not
+    // in the thumbnail format: there the attention warps' key rebuild is the
+    // bound, and the scan warp keeps ahead of them alone.
+    if (!dense && !kTR) {
+      bool failed = false;
+      uint64_t t0 = global_timer_ns();
+      while (!__shfl_sync(kFull, lane == 0 ? seq[st] == it : 0, 0)) {
+        const int e = claim_scan_entry<NSA>(sh, full_a, nref + nbs, true, lane);
+        if (e == -1) break;  // every entry is taken: wait for the item alone
+        if (e >= 0) {
+          const int jb = scan_block_index(e, nref, nb, j0);
+          if (!score_scan_entry_helper<T, G, F>(sh, scan_ring, full_a, empty_a, e, min(T, len - jb * T), lane,
+                                                p.wait_limit_ns)) {
+            failed = true;
+            break;
+          }
+          t0 = global_timer_ns();
+        } else if (global_timer_ns() - t0 > p.wait_limit_ns) {
+          failed = true;
+          break;
+        } else {
+          __nanosleep(20);
+        }
+      }
+      if (failed) {
+        raise_timeout(p, ctrl);
+        break;
+      }
+    }
     // Items go to the attention warps round-robin, so a warp can reach item
     // `it` before the stage's previous fill (another warp's item) has landed;
     // a parity wait could then match that older phase.  The producer writes
@@ -978,10 +1180,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   named_barrier(1, kAttnThreads);
-  const size_t unit = row * p.nsplit_max + split;
-  float *part = p.partials + unit * G * kPartialStride;
+  const size_t unit = (row * p.nsplit_max + split) * R + part;
+  float *part_out = p.partials + unit * G * kPartialStride;
   const bool unit_ok =
-      FFD_IN_BOUNDS(p, unit < static_cast<size_t>(p.batch) * p.num_kv_heads * p.nsplit_max && split < p.nsplit_max);
+      FFD_IN_BOUNDS(p, unit < static_cast<size_t>(p.batch) * p.num_kv_heads * p.nsplit_max * R && split < p.nsplit_max);
   for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kAttnThreads) {
     const int h = idx >> 7, c = idx & 127;
     float M = -INFINITY;
@@ -998,26 +1200,27 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     if (unit_ok) {
-      part[h * kPartialStride + c] = A;
+      part_out[h * kPartialStride + c] = A;
       if (c == 0) {
-        part[h * kPartialStride + 128] = M;
-        part[h * kPartialStride + 129] = L;
+        part_out[h * kPartialStride + 128] = M;
+        part_out[h * kPartialStride + 129] = L;
       }
     }
   }
-  if (static_cast<int>(threadIdx.x) < p.split_words) {
+  // (every part of a split holds the same selection: part 0 writes it)
+  if (part == 0 && static_cast<int>(threadIdx.x) < p.split_words) {
     uint32_t bits = keepbits[threadIdx.x];
     if (dense) {  // every valid block of the split
       const int lo = 32 * threadIdx.x;
       bits = lo >= nbs ? 0u : (nbs - lo >= 32 ? kFull : ((1u << (nbs - lo)) - 1u));
     }
-    if (unit_ok) p.split_bits[unit * p.split_words + threadIdx.x] = bits;
+    if (unit_ok) p.split_bits[(row * p.nsplit_max + split) * p.split_words + threadIdx.x] = bits;
     // splits of a multiple of 32 blocks own whole mask words: write them here
     // rather than gather them in the final merge
     if (!p.partials_only && (p.split_blocks & 31) == 0 && (j0 >> 5) + static_cast<int>(threadIdx.x) < p.mask_words)
       p.mask[row * p.mask_words + (j0 >> 5) + threadIdx.x] = bits;
   }
-  if (!p.partials_only && (p.split_blocks & 31) == 0 && split == nsplit - 1) {
+  if (!p.partials_only && (p.split_blocks & 31) == 0 && split == nsplit - 1 && part == 0) {
     // the last split also clears the words past its range
     for (int w = ((j0 + p.split_blocks) >> 5) + static_cast<int>(threadIdx.x); w < p.mask_words; w += kAttnThreads)
       p.mask[row * p.mask_words + w] = 0u;
@@ -1028,7 +1231,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // merges, its loads ordered after every other split's by the same add.
   named_barrier(1, kAttnThreads);
   if (threadIdx.x == 0)
-    ctrl[2] = atomic_add_acq_rel_gpu(&p.counters[row], 1u) == static_cast<uint32_t>(nsplit - 1) ? 1 : 0;
+    ctrl[2] = atomic_add_acq_rel_gpu(&p.counters[row], 1u) == static_cast<uint32_t>(nsplit * R - 1) ? 1 : 0;
   named_barrier(1, kAttnThreads);
   if (!ctrl[2]) return;
 
@@ -1040,17 +1243,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   // (m1, l1, o1) + (m2, l2, o2) = (M, l1 2^(m1 - M) + l2 2^(m2 - M),
   // o1 2^(m1 - M) + o2 2^(m2 - M)), M = max(m1, m2).  A split that kept no
   // token has m = -inf and is skipped.
-  const float *row_parts = p.partials + row * p.nsplit_max * G * kPartialStride;
+  const float *row_parts = p.partials + row * p.nsplit_max * R * G * kPartialStride;
+  const int nunits = nsplit * R;  // the split partials, R per split
   constexpr int kChunk = 16;
   for (int h = warp; h < G; h += kAttnWarps) {
     float M = -INFINITY, L = 0.0f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < nsplit; s0 += kChunk) {
+    for (int s0 = 0; s0 < nunits; s0 += kChunk) {
       float ms[kChunk], ls[kChunk];
       float4 v[kChunk];
 #pragma unroll
       for (int u = 0; u < kChunk; ++u) {
-        if (s0 + u < nsplit) {
+        if (s0 + u < nunits) {
           const float *ps = row_parts + ((s0 + u) * G + h) * kPartialStride;
           ms[u] = __ldcg(ps + 128);
           ls[u] = __ldcg(ps + 129);
@@ -1102,11 +1306,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <int T, int F>
-size_t smem_bytes_tf(int split_blocks) {
-  const int split_words = (split_blocks + 31) / 32;
-  return 1024 + SmemLayout<T, F>::kKeep + 4 * static_cast<size_t>((split_words + 3) & ~3) +
+constexpr size_t smem_bytes_tf(int split_blocks) {
+  return 1024 + SmemLayout<T, F>::kKeep + 4 * static_cast<size_t>((((split_blocks + 31) / 32) + 3) & ~3) +
          2 * static_cast<size_t>((split_blocks + 7) & ~7);
 }
+
+// Two CTAs per SM (the launch bounds) need each CTA's dynamic shared memory
+// within half of the SM's 228 KiB, less 1 KiB the hardware keeps per CTA.
+constexpr size_t kSmemPerCta2 = (228 * 1024) / 2 - 1024;
+static_assert(smem_bytes_tf<64, kFormatInt4>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<128, kFormatInt4>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<64, kFormatThumbResid>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<128, kFormatThumbResid>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
 
 // Raise the kernel's dynamic shared memory cap once per device, to the
 // largest split this library accepts, so later launches (and graph captures)

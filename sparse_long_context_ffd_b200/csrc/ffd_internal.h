@@ -64,6 +64,10 @@ struct DecodeParams {
   // context sharding: write the split partials and bits only (no final merge;
   // out and mask unused)
   int32_t partials_only;
+  // CTAs per split (grid.x = nsplit_max * parts): each scans the whole split
+  // and attends over the kept blocks at kept-list positions = its index mod
+  // parts, writing its own partial (partials [..][nsplit_max][parts][G][..])
+  int32_t parts;
   // limit of the pipeline and queue waits (the drains of the kernel's own
   // copies always use kWaitLimitNs)
   uint64_t wait_limit_ns;
@@ -92,11 +96,19 @@ struct QuantizeParams {
 // Workspace carve-up (byte offsets), identical on host and device.
 struct WorkspaceLayout {
   size_t err, counters, split_bits, partials, total;
-  int32_t nsplit_max, split_words;
+  int32_t nsplit_max, split_words, parts;
 };
 
+// CTAs per split for a shape: the largest power of two up to 8 (and up to the
+// split size) for which batch * kv-heads * splits * parts still fits in one
+// wave of two CTAs on each of a B200's 148 SMs.
+int32_t parts_per_split(int32_t batch, int32_t num_kv_heads, int32_t capacity, int32_t block_size,
+                        int32_t split_blocks);
+
+// parts: CTAs per split (the partials hold one slot per part).
 WorkspaceLayout workspace_layout(int32_t batch, int32_t num_kv_heads, int32_t group,
-                                 int32_t capacity, int32_t block_size, int32_t split_blocks);
+                                 int32_t capacity, int32_t block_size, int32_t split_blocks,
+                                 int32_t parts = 1);
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format);
 

@@ -60,7 +60,14 @@ def test_buffer_sizes(B, Hq, Hkv, cap, T, S):
     assert ffd.thumb_bytes(s) == B * Hkv * cap * 32
     assert ffd.residual_bytes(s) == B * Hkv * cap * 128
     nsplit = math.ceil(cap // T / S)
-    partials = B * Hkv * nsplit * (Hq // Hkv) * 132 * 4
+    # CTAs per split (documented with ffd_decode_workspace_bytes): the largest
+    # power of two up to 8 and up to S for which B * Hkv * nsplit * R <= 296
+    R = 1
+    while R < 8 and 2 * R <= S and B * Hkv * nsplit * 2 * R <= 296:
+        R *= 2
+    assert R == {(1, 4096): 8, (4, 32768): 1, (1, 131072): 1, (1, 262144): 1, (16, 65536): 1,
+                 (3, 640): 2}[(B, cap)]
+    partials = B * Hkv * nsplit * R * (Hq // Hkv) * 132 * 4
     ws = ffd.decode_workspace_bytes(s)
     assert ws >= partials + B * Hkv * 4 + 4 and ws % 256 == 0
     assert ws <= partials + 4 * 256 + B * Hkv * 4 + B * Hkv * nsplit * math.ceil(S / 32) * 4
