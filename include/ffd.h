@@ -104,7 +104,10 @@ size_t ffd_mask_words(const ffd_shape *shape);
  * power of two up to 8 and up to S with B * Hkv * ceil(nblk / S) * R <= 296,
  * two CTAs on each of a B200's 148 SMs): each scans the whole split, so all
  * take the same selection with no exchange, and attends over every R-th kept
- * block; the partials then hold R slots per split.  0 for an invalid shape. */
+ * block; the partials then hold R slots per split.  The selection bits a call
+ * leaves in the workspace also steer how the next call on it spreads the
+ * selector's work over its warps (never what it computes).  0 for an invalid
+ * shape. */
 size_t ffd_decode_workspace_bytes(const ffd_shape *shape);
 
 /* Zero a workspace (cudaMemsetAsync on the stream).  Call once after

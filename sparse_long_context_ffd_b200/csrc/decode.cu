@@ -94,27 +94,30 @@ struct KvGeom<kFormatThumbResid> {
   static constexpr int kStages = 6;
 };
 
-template <int T, int F>
+// C: the cooperative selector (several warps score scan entries).  Then the
+// ring has as many stages as fit beside the K/V ring with two CTAs per SM,
+// since several warps hold stages at once; with the scan warp alone, fewer.
+template <int T, int F, bool C>
 struct ScanGeom {
   static constexpr int kRowBytes = F == kFormatThumbResid ? kThumbRowBytes : kPackedRowBytes;
   static constexpr int kStageBytes = T * kRowBytes + kScaleRowBytes;
-  // As many stages as fit beside the K/V ring with two CTAs per SM: several
-  // warps score entries at once, and each holds its stage while it reads it.
-  static constexpr int kStages = F == kFormatThumbResid ? (T == 64 ? 9 : 5) : (T == 64 ? 6 : 3);
+  static constexpr int kStages = C ? (F == kFormatThumbResid ? (T == 64 ? 9 : 5) : (T == 64 ? 6 : 3))
+                                   : (F == kFormatThumbResid ? 2 : 1) * (T == 64 ? 4 : 2);
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
 };
 
-template <int T, int F>
+template <int T, int F, bool C>
 struct SmemLayout {
   static constexpr int NKV = KvGeom<F>::kStages;
   static constexpr int kKvRing = 0;
   static constexpr int kScanRing = NKV * KvGeom<F>::kStageBytes;
-  static constexpr int kBars = kScanRing + ScanGeom<T, F>::kRingBytes;
-  static constexpr int kNumBars = 2 * ScanGeom<T, F>::kStages + 2 * NKV;
+  static constexpr int kBars = kScanRing + ScanGeom<T, F, C>::kRingBytes;
+  static constexpr int kNumBars = 2 * ScanGeom<T, F, C>::kStages + 2 * NKV;
   static constexpr int kMeta = kBars + 8 * kNumBars;  // int [NKV] token offsets
   static constexpr int kSeq = kMeta + 4 * NKV;        // int [NKV] item indices
-  // qcount, sel_done, is_last, abort, requant_done, scan claim, scan decided
+  // qcount, sel_done, is_last, abort, requant_done, scan claim, scan decided,
+  // attention warps help the scan
   static constexpr int kCtrl = (kSeq + 4 * NKV + 15) / 16 * 16;
   static constexpr int kScanSeq = kCtrl + 32;                // int [NSA] scan entry per stage
   static constexpr int kSlotSeq = kScanSeq + 4 * kScanSlots;  // int [kScanSlots] entry per slot
@@ -123,7 +126,7 @@ struct SmemLayout {
   static constexpr int kRequant = kQRows + 8 * kHeadDim * 2;  // re-quantisation scratch (attention warps)
   static constexpr int kKeep = kRequant + kRequantScratchBytes;  // u32 [split_words]
   // queue of kept block indices (u16 [split_blocks]) follows keep bits
-  static_assert(ScanGeom<T, F>::kStages <= kScanSlots, "one sequence word per scan stage");
+  static_assert(ScanGeom<T, F, C>::kStages <= kScanSlots, "one sequence word per scan stage");
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -462,11 +465,11 @@ __device__ __forceinline__ int claim_scan_entry(const ScanShared &sh, uint64_t *
 // producer's sequence word, then the stage's fill, both bounded), fold the
 // query with the block's scales, scan, release the stage.  s0, s1: the
 // scores of heads 2 t4 and 2 t4 + 1 (every lane).  False if a wait ran out.
-template <int T, int G, int F>
+template <int T, int G, int F, bool C>
 __device__ __forceinline__ bool score_scan_entry(const ScanShared &sh, uint8_t *scan_ring, uint64_t *full_a,
                                                  uint64_t *empty_a, int e, int valid_rows, int lane,
                                                  uint64_t limit_ns, float &s0, float &s1) {
-  using SG = ScanGeom<T, F>;
+  using SG = ScanGeom<T, F, C>;
   using SF = ScanFold<G, F>;
   constexpr int NSA = SG::kStages;
   const int st = e % NSA;
@@ -511,18 +514,21 @@ __device__ __noinline__ bool score_scan_entry_helper(const ScanShared &sh, uint8
                                                      uint64_t *empty_a, int e, int valid_rows, int lane,
                                                      uint64_t limit_ns) {
   float s0, s1;
-  if (!score_scan_entry<T, G, F>(sh, scan_ring, full_a, empty_a, e, valid_rows, lane, limit_ns, s0, s1))
+  if (!score_scan_entry<T, G, F, true>(sh, scan_ring, full_a, empty_a, e, valid_rows, lane, limit_ns, s0, s1))
     return false;
   publish_scan_scores(sh, e, s0, s1, lane);
   return true;
 }
 
-template <int T, int G, int F>
+// C: the cooperative selector (the attention warps score scan entries while
+// they wait for K/V); launched for the int4 format's sparse steps.  Without it
+// (dense mode, the thumbnail format) the scan warp scores every entry itself.
+template <int T, int G, int F, bool C>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
-  using SG = ScanGeom<T, F>;
-  using SL = SmemLayout<T, F>;
+  using SG = ScanGeom<T, F, C>;
+  using SL = SmemLayout<T, F, C>;
   using KG = KvGeom<F>;
   constexpr bool kTR = F == kFormatThumbResid;
   constexpr int NSA = SG::kStages;
@@ -600,16 +606,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&empty_b[s], 1);
       seq[s] = -1;
     }
-    for (int c = 0; c < 7; ++c) ctrl[c] = 0;
+    for (int c = 0; c < 8; ++c) ctrl[c] = 0;
     for (int s = 0; s < NSA; ++s) sh.scan_seq[s] = -1;
     for (int s = 0; s < kScanSlots; ++s) sh.slot_seq[s] = -1;
     fence_mbar_init();
   }
   for (int w = threadIdx.x; w < p.split_words; w += blockDim.x) keepbits[w] = 0u;
-  // the query group, for every warp that scores scan entries
-  for (int i = threadIdx.x; i < G * kHeadDim / 8; i += blockDim.x)
-    reinterpret_cast<uint4 *>(smem + SL::kQRows)[i] = reinterpret_cast<const uint4 *>(
-        p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim)[i];
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
@@ -632,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int scan_total = dense ? 0 : nref + nbs;
     int sc_next = 0;                // scan tiles issued
     int it_next = 0;                // attention stages issued (items + end markers)
-    int q_ptr = 0, sub = 0;         // position in the kept-block list
+    int q_ptr = part, sub = 0;      // position in the kept-block list (this part's: part + k R)
     int ends_sent = 0;
     uint64_t idle_since = 0;
     // copies that read the last block's re-quantised data wait for the
@@ -677,14 +679,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool sel_done = dense || ld_acquire_cta(&ctrl[1]) != 0;
       const int avail = dense ? nbs : ld_acquire_cta(&ctrl[0]);
       while (q_ptr < avail) {
-        if (q_ptr % R != part) {  // another part's block
-          ++q_ptr;
-          continue;
-        }
         const int j = dense ? q_ptr : static_cast<int>(queue[q_ptr]);
         const int tok = (j0 + j) * T + sub * kKvTok;
         if (sub >= kSubPerBlock || tok >= len) {
-          ++q_ptr;
+          q_ptr += R;  // this part's next kept block
           sub = 0;
           continue;
         }
@@ -787,9 +785,77 @@ __global__ void __launch_bounds__(kThreads, 2)
         ++qn;
       }
     };
+    const int total = nref + nbs;
+    // Cooperative selector: the attention warps help the scan unless this
+    // CTA's share of the split's kept blocks in the previous call on this
+    // workspace (the split's selection bits are still there, and a part
+    // attends over 1 / R of them) was at least 3/4 of the split: then the
+    // attention warps are the bound and the scan warp keeps ahead alone.
+    // This only spreads the work; the selection and the output do not depend
+    // on it.  Decided here, after the pipeline has started, and published
+    // (with the query group copied for the helpers) in ctrl[7].
+    bool help = false;
+    if constexpr (C) {
+      // (both loads in flight together: the query group, 16 bytes x G x 16
+      // over the lanes, and the split's previous bits)
+      constexpr int kQv = (G * kHeadDim / 8 + 31) / 32;
+      uint4 qrow[kQv];
+      const uint4 *qsrc = reinterpret_cast<const uint4 *>(
+          p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G) * kHeadDim);
+#pragma unroll
+      for (int k = 0; k < kQv; ++k)
+        if (lane + 32 * k < G * kHeadDim / 8) qrow[k] = qsrc[lane + 32 * k];
+      int prev = 0;
+      for (int w = lane; w < p.split_words; w += 32)
+        prev += __popc(__ldcg(p.split_bits + (row * p.nsplit_max + split) * p.split_words + w));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) prev += __shfl_xor_sync(kFull, prev, off);
+      help = 4 * prev < 3 * nbs * R;  // (a part attends over 1 / R of the kept blocks)
+      if (help) {
+#pragma unroll
+        for (int k = 0; k < kQv; ++k)
+          if (lane + 32 * k < G * kHeadDim / 8) reinterpret_cast<uint4 *>(smem + SL::kQRows)[lane + 32 * k] = qrow[k];
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          ctrl[7] = 1;
+        }
+      }
+    }
+    if (!help) {
+      // the scan warp alone: every entry in order, the query in registers
+      using SF = ScanFold<G, F>;
+      uint32_t qv[SF::NC / 2];
+      SF::load_pairs(p.q + (static_cast<size_t>(b) * num_q_heads + static_cast<size_t>(g) * G + gid % G) *
+                               kHeadDim + 32 * t4,
+                     SF::part(gid), qv);
+      for (int e = 0; e < total; ++e) {
+        const int st = e % NSA;
+        if (!mbar_wait(&full_a[st], static_cast<uint32_t>(e / NSA) & 1u, p.wait_limit_ns)) {
+          raise_timeout(p, ctrl);
+          break;
+        }
+        const int jb = scan_block_index(e, nref, nb, j0);
+        const uint8_t *tile = scan_ring + st * SG::kStageBytes;
+        uint32_t bq[8];
+        int sq, best0, best1;
+        float am, s0, s1;
+        fold_block<G, F>(reinterpret_cast<const uint16_t *>(tile + T * SG::kRowBytes), qv, lane, bq, sq, am);
+        block_best<T, F>(tile, bq, min(T, len - jb * T), lane, best0, best1);
+        block_scores<F>(best0, best1, sq, am, lane, s0, s1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_a[st]);
+        decide(e, s0, s1);
+        if (__shfl_sync(kFull, lane == 0 ? ctrl[3] : 0, 0)) break;
+      }
+      if (lane == 0) {
+        __threadfence_block();
+        ctrl[1] = 1;
+      }
+      return;
+    }
     // score entries (the attention warps help while they wait for K/V) and
     // decide them in block order
-    const int total = nref + nbs;
     int decided = 0;
     uint64_t idle_since = 0;
     while (true) {
@@ -815,8 +881,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (e >= 0) {
         const int jb = scan_block_index(e, nref, nb, j0);
         float s0, s1;
-        if (!score_scan_entry<T, G, F>(sh, scan_ring, full_a, empty_a, e, min(T, len - jb * T), lane,
-                                       p.wait_limit_ns, s0, s1)) {
+        if (!score_scan_entry<T, G, F, C>(sh, scan_ring, full_a, empty_a, e, min(T, len - jb * T), lane,
+                                          p.wait_limit_ns, s0, s1)) {
           raise_timeout(p, ctrl);
           break;
         }
@@ -960,10 +1026,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int it = warp;; it += kAttnWarps) {
     const int st = it % NKV;
     // Until item `it` is published, score scan entries whose tiles have
-    // landed (the selector's work, decided in order by the scan warp).  Not
-    // in the thumbnail format: there the attention warps' key rebuild is the
-    // bound, and the scan warp keeps ahead of them alone.
-    if (!dense && !kTR) {
+    // landed (the selector's work, decided in order by the scan warp).
+    if (C && __shfl_sync(kFull, lane == 0 ? ctrl[7] : 0, 0) != 0) {  // (one value for the warp)
       bool failed = false;
       uint64_t t0 = global_timer_ns();
       while (!__shfl_sync(kFull, lane == 0 ? seq[st] == it : 0, 0)) {
@@ -1305,46 +1369,70 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) p.counters[row] = 0u;
 }
 
-template <int T, int F>
+template <int T, int F, bool C>
 constexpr size_t smem_bytes_tf(int split_blocks) {
-  return 1024 + SmemLayout<T, F>::kKeep + 4 * static_cast<size_t>((((split_blocks + 31) / 32) + 3) & ~3) +
+  return 1024 + SmemLayout<T, F, C>::kKeep + 4 * static_cast<size_t>((((split_blocks + 31) / 32) + 3) & ~3) +
          2 * static_cast<size_t>((split_blocks + 7) & ~7);
 }
 
 // Two CTAs per SM (the launch bounds) need each CTA's dynamic shared memory
 // within half of the SM's 228 KiB, less 1 KiB the hardware keeps per CTA.
 constexpr size_t kSmemPerCta2 = (228 * 1024) / 2 - 1024;
-static_assert(smem_bytes_tf<64, kFormatInt4>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
-static_assert(smem_bytes_tf<128, kFormatInt4>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
-static_assert(smem_bytes_tf<64, kFormatThumbResid>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
-static_assert(smem_bytes_tf<128, kFormatThumbResid>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<64, kFormatInt4, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<128, kFormatInt4, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<64, kFormatThumbResid, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<128, kFormatThumbResid, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
 
 // Raise the kernel's dynamic shared memory cap once per device, to the
 // largest split this library accepts, so later launches (and graph captures)
 // need no attribute call.
-template <int T, int G, int F>
-cudaError_t configure_tgf() {
+template <int T, int G, int F, bool C>
+cudaError_t configure_tgfc() {
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
   if (bit == 0 || (configured.load(std::memory_order_acquire) & bit) == 0) {
-    e = cudaFuncSetAttribute(decode_kernel<T, G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes_tf<T, F>(FFD_MAX_SPLIT_BLOCKS)));
+    e = cudaFuncSetAttribute(decode_kernel<T, G, F, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes_tf<T, F, C>(FFD_MAX_SPLIT_BLOCKS)));
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   return cudaSuccess;
 }
 
+// The variants of one (T, G, F): the int4 format has both selectors, the
+// thumbnail format only the scan warp's.
+// The cooperative selector is built for the int4 format's 64-token blocks
+// (at 128 tokens its registers spill); dense mode has no selector.
+template <int T, int F>
+constexpr bool kHasCoop = F == kFormatInt4 && T == 64;
+
+template <int T, int G, int F>
+cudaError_t configure_tgf() {
+  cudaError_t e = configure_tgfc<T, G, F, false>();
+  if (e == cudaSuccess && kHasCoop<T, F>) e = configure_tgfc<T, G, F, kHasCoop<T, F>>();
+  return e;
+}
+
+template <int T, int G, int F, bool C>
+cudaError_t launch_tgfc(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
+                        cudaStream_t stream) {
+  cudaError_t e = configure_tgfc<T, G, F, C>();
+  if (e != cudaSuccess) return e;
+  const size_t smem = smem_bytes_tf<T, F, C>(p.split_blocks);
+  decode_kernel<T, G, F, C><<<grid, kThreads, smem, stream>>>(p, tk, tv);
+  return cudaGetLastError();
+}
+
+// The cooperative selector is built for the int4 format's 64-token blocks
+// (at 128 tokens its registers spill); dense mode has no selector.
 template <int T, int G, int F>
 cudaError_t launch_tgf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
-                       size_t smem, cudaStream_t stream) {
-  cudaError_t e = configure_tgf<T, G, F>();
-  if (e != cudaSuccess) return e;
-  decode_kernel<T, G, F><<<grid, kThreads, smem, stream>>>(p, tk, tv);
-  return cudaGetLastError();
+                       cudaStream_t stream) {
+  if (kHasCoop<T, F> && !p.dense) return launch_tgfc<T, G, F, kHasCoop<T, F>>(p, tk, tv, grid, stream);
+  return launch_tgfc<T, G, F, false>(p, tk, tv, grid, stream);
 }
 
 template <int T, int F>
@@ -1360,21 +1448,21 @@ cudaError_t configure_tf(int group) {
 
 template <int T, int F>
 cudaError_t launch_tf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int group,
-                      dim3 grid, size_t smem, cudaStream_t stream) {
+                      dim3 grid, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_tgf<T, 1, F>(p, tk, tv, grid, smem, stream);
-    case 2: return launch_tgf<T, 2, F>(p, tk, tv, grid, smem, stream);
-    case 4: return launch_tgf<T, 4, F>(p, tk, tv, grid, smem, stream);
-    case 8: return launch_tgf<T, 8, F>(p, tk, tv, grid, smem, stream);
+    case 1: return launch_tgf<T, 1, F>(p, tk, tv, grid, stream);
+    case 2: return launch_tgf<T, 2, F>(p, tk, tv, grid, stream);
+    case 4: return launch_tgf<T, 4, F>(p, tk, tv, grid, stream);
+    case 8: return launch_tgf<T, 8, F>(p, tk, tv, grid, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int F>
 cudaError_t launch_f(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int block_size,
-                     int group, dim3 grid, size_t smem, cudaStream_t stream) {
-  if (block_size == 64) return launch_tf<64, F>(p, tk, tv, group, grid, smem, stream);
-  if (block_size == 128) return launch_tf<128, F>(p, tk, tv, group, grid, smem, stream);
+                     int group, dim3 grid, cudaStream_t stream) {
+  if (block_size == 64) return launch_tf<64, F>(p, tk, tv, group, grid, stream);
+  if (block_size == 128) return launch_tf<128, F>(p, tk, tv, group, grid, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -1391,11 +1479,12 @@ __global__ void bounds_selftest_kernel(DecodeParams p) {
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format) {
   (void)group;
+  // the larger of a format's variants (the cooperative one for int4)
   if (format == kFormatThumbResid)
-    return block_size == 64 ? smem_bytes_tf<64, kFormatThumbResid>(split_blocks)
-                            : smem_bytes_tf<128, kFormatThumbResid>(split_blocks);
-  return block_size == 64 ? smem_bytes_tf<64, kFormatInt4>(split_blocks)
-                          : smem_bytes_tf<128, kFormatInt4>(split_blocks);
+    return block_size == 64 ? smem_bytes_tf<64, kFormatThumbResid, false>(split_blocks)
+                            : smem_bytes_tf<128, kFormatThumbResid, false>(split_blocks);
+  return block_size == 64 ? smem_bytes_tf<64, kFormatInt4, true>(split_blocks)
+                          : smem_bytes_tf<128, kFormatInt4, false>(split_blocks);
 }
 
 cudaError_t prepare_decode(int block_size, int group, int format) {
@@ -1409,10 +1498,11 @@ cudaError_t prepare_decode(int block_size, int group, int format) {
 cudaError_t launch_decode(const DecodeParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
                           int block_size, int group, int format, dim3 grid, size_t smem_bytes,
                           cudaStream_t stream) {
+  (void)smem_bytes;  // each variant's own size is used
   if (format == kFormatThumbResid)
-    return launch_f<kFormatThumbResid>(p, tmap_k, tmap_v, block_size, group, grid, smem_bytes, stream);
+    return launch_f<kFormatThumbResid>(p, tmap_k, tmap_v, block_size, group, grid, stream);
   if (format == kFormatInt4)
-    return launch_f<kFormatInt4>(p, tmap_k, tmap_v, block_size, group, grid, smem_bytes, stream);
+    return launch_f<kFormatInt4>(p, tmap_k, tmap_v, block_size, group, grid, stream);
   return cudaErrorInvalidValue;
 }
 
