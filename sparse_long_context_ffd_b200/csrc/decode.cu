@@ -1027,11 +1027,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int st = it % NKV;
     // Until item `it` is published, score scan entries whose tiles have
     // landed (the selector's work, decided in order by the scan warp).
-    if (C && __shfl_sync(kFull, lane == 0 ? ctrl[7] : 0, 0) != 0) {  // (one value for the warp)
+    // (The scan warp publishes whether to help shortly after the start, so
+    // the flag is read on every turn of the wait, one value for the warp.)
+    if (C && !dense) {
       bool failed = false;
       uint64_t t0 = global_timer_ns();
       while (!__shfl_sync(kFull, lane == 0 ? seq[st] == it : 0, 0)) {
-        const int e = claim_scan_entry<NSA>(sh, full_a, nref + nbs, true, lane);
+        const bool help = __shfl_sync(kFull, lane == 0 ? ctrl[7] : 0, 0) != 0;
+        const int e = help ? claim_scan_entry<NSA>(sh, full_a, nref + nbs, true, lane) : -2;
         if (e == -1) break;  // every entry is taken: wait for the item alone
         if (e >= 0) {
           const int jb = scan_block_index(e, nref, nb, j0);

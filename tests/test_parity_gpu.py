@@ -371,3 +371,36 @@ def test_full_config_pseudo_max(name, delta, ref):
     kept = sum(int(oracle.mask_to_blocks(mask[b, g], nblk).sum())
                for b in range(w.batch) for g in range(w.num_kv_heads))
     print(tag, "kept", kept, "max-abs", mx, "mean-abs", mean)
+
+
+# ---------------------------- concentrated attention, small kept fractions --
+
+@pytest.mark.parametrize("batch", [4, 1], ids=["one_cta_per_split", "several_ctas_per_split"])
+def test_kept_fraction_and_call_history_do_not_change_results(batch):
+    # The controlled-sparsity workloads (n of every 64 blocks raised above the
+    # rest) at a 32K context: B4 x 8 kv-heads gives one CTA per split, B1 eight.
+    # Calls alternate between 1/64 and all blocks kept on the same workspace,
+    # so the cooperative selector's per-call switch (from the previous call's
+    # selection bits) is exercised both ways; every call must match the oracle.
+    from gpu_util import bf16_to_np_f32
+    cases = []
+    for name in ("rho1of64", "rho1"):
+        w = fw.scaled_workload(fw.WORKLOADS[name], batch=batch, capacity=32768, context=32768)
+        inp = fw.make_inputs(w)
+        packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+        want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales,
+                                               inp["lengths"], w.block_size, w.split_blocks, w.delta)
+        cases.append((name, w, inp, want_out, want_mask))
+    ws = None
+    for name, w, inp, want_out, want_mask in cases + cases + cases[:1]:
+        gc = GpuCase(w, inp)
+        if ws is None:
+            ws = gc.bufs.workspace
+        gc.quantize(0)
+        ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
+                      w.delta, gc.bufs.out, gc.bufs.mask, ws, requant_last=True)
+        torch.cuda.synchronize()
+        mask = gc.bufs.mask.cpu().numpy().view(np.uint32)
+        assert_mask_equal(mask, want_mask, f"{name} B{batch}")
+        assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, f"{name} B{batch}")
+        assert ffd.check_device_status(ws) == 0
