@@ -404,3 +404,27 @@ def test_kept_fraction_and_call_history_do_not_change_results(batch):
         assert_mask_equal(mask, want_mask, f"{name} B{batch}")
         assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, f"{name} B{batch}")
         assert ffd.check_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("context", [16384, 32768])
+@pytest.mark.parametrize("delta", [3.0, 0.5, INF])
+def test_short_context_shares_splits_between_ctas(context, delta):
+    # One sequence of the long-context shape at 16K / 32K: 32 / 64 (split,
+    # kv-head) units, so 8 / 4 CTAs share each split (each scans all of it and
+    # attends over every 8th / 4th kept block); the fused step against the
+    # oracle, mask bit-exact.
+    from gpu_util import bf16_to_np_f32
+    w = fw.scaled_workload(fw.WORKLOADS["long128k"], capacity=context, context=context)
+    inp = fw.make_inputs(w)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales,
+                                           inp["lengths"], w.block_size, w.split_blocks, delta)
+    gc = GpuCase(w, inp)
+    gc.quantize(0)
+    for _ in range(2):  # (the second call sees the first one's selection bits)
+        ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths,
+                      delta, gc.bufs.out, gc.bufs.mask, gc.bufs.workspace, requant_last=True)
+        torch.cuda.synchronize()
+        assert_mask_equal(gc.bufs.mask.cpu().numpy().view(np.uint32), want_mask, f"{context} {delta}")
+        assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, f"{context} {delta}")
+    assert ffd.check_device_status(gc.bufs.workspace) == 0

@@ -287,3 +287,19 @@ def test_decode_tr_full_config(name, deltas):
         kept = sum(int(oracle.mask_to_blocks(mask[b, g], nblk).sum())
                    for b in range(w.batch) for g in range(w.num_kv_heads))
         print("tr", name, delta, "kept", kept, "max-abs", mx, "mean-abs", mean)
+
+
+@pytest.mark.parametrize("delta", [3.0, INF])
+def test_decode_tr_short_context_shares_splits_between_ctas(delta):
+    # one 16K sequence of the long-context shape: 8 CTAs share each split
+    w = fw.scaled_workload(fw.WORKLOADS["long128k"], capacity=16384, context=16384)
+    inp = fw.make_inputs(w)
+    thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], w.block_size)
+    want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales, inp["lengths"],
+                                              w.block_size, w.split_blocks, delta)
+    tc = TrCase(w, inp)
+    tc.quantize(0)
+    out, mask = tc.decode(delta, requant_last=True)
+    assert_mask_equal(mask, want_mask, f"tr 16K {delta}")
+    assert_output_close(out, want_out, f"tr 16K {delta}")
+    assert ffd.check_device_status(tc.bufs.workspace) == 0
