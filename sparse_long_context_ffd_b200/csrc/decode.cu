@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 
@@ -72,19 +73,23 @@ constexpr int kRequantScratchBytes = (kAttnWarps + 1) * kHeadDim * 4;
 // uses slot e % kScanSlots, so at most kScanSlots entries are claimed ahead of
 // the decision frontier.
 constexpr int kScanSlots = 16;
+// Thumbnail format: longest split (tokens) whose sparse steps load the
+// attention stages' thumbnail rows and scale rows from L2 (KvGeom).
+constexpr int kTrL2MaxSplitTokens = 4096;
 
-// One attention stage (kKvTok tokens of one kept block) per key format.
-template <int F>
+// One attention stage (kKvTok tokens of one kept block) per key format and
+// variant (C: the sparse-step variant, below).
+template <int F, bool C>
 struct KvGeom;
-template <>
-struct KvGeom<kFormatInt4> {  // K lo, K hi, V lo, V hi (bf16, 128-byte swizzle): 16 KiB
+template <bool C>
+struct KvGeom<kFormatInt4, C> {  // K lo, K hi, V lo, V hi (bf16, 128-byte swizzle): 16 KiB
   static constexpr int kVOffset = 2 * kKvHalfBytes;
   static constexpr int kTx = 4 * kKvHalfBytes;
   static constexpr int kStageBytes = kTx;
   static constexpr int kStages = 5;
 };
 template <>
-struct KvGeom<kFormatThumbResid> {
+struct KvGeom<kFormatThumbResid, false> {
   // residual rows (128 B, 128-byte swizzle) | V lo | V hi | thumbnail rows | scale row
   static constexpr int kVOffset = kKvTok * kResidRowBytes;
   static constexpr int kThumbOffset = kVOffset + 2 * kKvHalfBytes;
@@ -93,25 +98,37 @@ struct KvGeom<kFormatThumbResid> {
   static constexpr int kStageBytes = (kTx + 1023) / 1024 * 1024;  // swizzled tiles stay 1 KiB aligned
   static constexpr int kStages = 6;
 };
+template <>
+struct KvGeom<kFormatThumbResid, true> {
+  // residual rows | V lo | V hi: 12 KiB.  The stage's thumbnail rows and scale
+  // row (1.25 KiB) stay out of it: in a sparse step with short splits the scan
+  // read them shortly before, so the attention warp loads them from L2 into
+  // registers while the stage is in flight.  No small copies per stage, and
+  // one stage more in the same shared memory.
+  static constexpr int kVOffset = kKvTok * kResidRowBytes;
+  static constexpr int kTx = kVOffset + 2 * kKvHalfBytes;
+  static constexpr int kStageBytes = kTx;
+  static constexpr int kStages = 7;
+};
 
-// C: the cooperative selector (several warps score scan entries).  Then the
-// ring has as many stages as fit beside the K/V ring with two CTAs per SM,
-// since several warps hold stages at once; with the scan warp alone, fewer.
+// With the cooperative selector (int4, C) the ring has as many stages as fit
+// beside the K/V ring with two CTAs per SM, since several warps hold stages at
+// once; with the scan warp alone, fewer.
 template <int T, int F, bool C>
 struct ScanGeom {
   static constexpr int kRowBytes = F == kFormatThumbResid ? kThumbRowBytes : kPackedRowBytes;
   static constexpr int kStageBytes = T * kRowBytes + kScaleRowBytes;
-  static constexpr int kStages = C ? (F == kFormatThumbResid ? (T == 64 ? 9 : 5) : (T == 64 ? 6 : 3))
-                                   : (F == kFormatThumbResid ? 2 : 1) * (T == 64 ? 4 : 2);
+  static constexpr int kStages = F == kFormatThumbResid ? 2 * (T == 64 ? 4 : 2)
+                                                        : (C ? (T == 64 ? 6 : 3) : (T == 64 ? 4 : 2));
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
 };
 
 template <int T, int F, bool C>
 struct SmemLayout {
-  static constexpr int NKV = KvGeom<F>::kStages;
+  static constexpr int NKV = KvGeom<F, C>::kStages;
   static constexpr int kKvRing = 0;
-  static constexpr int kScanRing = NKV * KvGeom<F>::kStageBytes;
+  static constexpr int kScanRing = NKV * KvGeom<F, C>::kStageBytes;
   static constexpr int kBars = kScanRing + ScanGeom<T, F, C>::kRingBytes;
   static constexpr int kNumBars = 2 * ScanGeom<T, F, C>::kStages + 2 * NKV;
   static constexpr int kMeta = kBars + 8 * kNumBars;  // int [NKV] token offsets
@@ -520,17 +537,60 @@ __device__ __noinline__ bool score_scan_entry_helper(const ScanShared &sh, uint8
   return true;
 }
 
-// C: the cooperative selector (the attention warps score scan entries while
-// they wait for K/V); launched for the int4 format's sparse steps.  Without it
-// (dense mode, the thumbnail format) the scan warp scores every entry itself.
+// Thumbnail format: keys are rebuilt from thumbnail + residual as k_hat =
+// s z / 254 with the integer z = 254 u - 381 + e (exact in f16).  The block's
+// scales go into the query instead: q'_c = f16(q_c s_c 2^E / 254), E per head
+// so that max |q'| is about 2^13 (no f16 overflow or underflow), and the scores
+// are scaled back by 2^-E in fp32.  qb: the lane's query pairs (channels
+// 32*t4 + 2i, +1 of head gid, i = 2ks + j at qb[ks][j]); scale4(w4): the lane's
+// scales of channels 32*t4 + 8*w4 .. +7.  Returns q' as f16 pairs in qh and
+// the logit scales of heads 2*t4, 2*t4 + 1 (every lane).
+template <typename ScaleFn>
+__device__ __forceinline__ void fold_query_tr(const uint32_t (&qb)[8][2], int t4, ScaleFn scale4, uint32_t (&qh)[16],
+                                              float &sc0, float &sc1) {
+  float fq[32];
+  float am = 0.0f;
+#pragma unroll
+  for (int w4 = 0; w4 < 4; ++w4) {
+    const uint4 sv = scale4(w4);
+    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = 4 * w4 + e;  // channel pair 32*t4 + 2i
+      const uint32_t qw = qb[i >> 1][i & 1];
+      fq[2 * i] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
+      fq[2 * i + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
+      am = fmaxf(am, fmaxf(fabsf(fq[2 * i]), fabsf(fq[2 * i + 1])));
+    }
+  }
+  am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
+  am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
+  const int ea = static_cast<int>((__float_as_uint(am) >> 23) & 0xFFu);
+  const int E = min(148 - ea, 126);  // am 2^E in [2^21, 2^22)
+  const float mult = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 + E) << 23) * (1.0f / 254.0f);
+  const float uns = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - E) << 23) * kScaleLog2;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) qh[i] = pack_f16x2(fq[2 * i] * mult, fq[2 * i + 1] * mult);
+  sc0 = __shfl_sync(kFull, uns, (2 * t4) << 2);
+  sc1 = __shfl_sync(kFull, uns, (2 * t4 + 1) << 2);
+}
+
+// C: the sparse-step variant for 64-token blocks.  int4 format: the
+// cooperative selector (the attention warps score scan entries while they wait
+// for K/V); without it (dense mode) the scan warp scores every entry itself.
+// Thumbnail format (splits of at most 4096 tokens): the attention stages leave
+// out the thumbnail rows and scale rows, which the attention warps load from
+// L2 (KvGeom); its selector is always the scan warp's.
 template <int T, int G, int F, bool C>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
   using SG = ScanGeom<T, F, C>;
   using SL = SmemLayout<T, F, C>;
-  using KG = KvGeom<F>;
+  using KG = KvGeom<F, C>;
   constexpr bool kTR = F == kFormatThumbResid;
+  constexpr bool kCoop = C && !kTR;  // the cooperative selector
+  constexpr bool kTrL2 = C && kTR;   // thumbnails and scales from L2
   constexpr int NSA = SG::kStages;
   constexpr int NKV = KG::kStages;
   constexpr int kSubPerBlock = T / kKvTok;
@@ -693,16 +753,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
         uint8_t *dst = kv_ring + st * KG::kStageBytes;
         meta[st] = tok;
+        if constexpr (kTrL2) __threadfence_block();  // (the computer reads meta once seq shows the item)
         seq[st] = it_next;
         mbar_arrive_expect_tx(&full_b[st], KG::kTx);
         const int y = row_tok0 + tok;
         if (FFD_IN_BOUNDS(p, tok >= 0 && tok + kKvTok <= p.capacity && row_ok)) {
           if constexpr (kTR) {
             tma_load_2d(dst, &tmap_k, 0, y, &full_b[st]);  // residual rows
-            bulk_g2s(dst + KG::kThumbOffset, src_p + static_cast<size_t>(tok) * kThumbRowBytes,
-                     kKvTok * kThumbRowBytes, &full_b[st]);
-            bulk_g2s(dst + KG::kScaleOffset, src_s + static_cast<size_t>(tok / T) * kHeadDim,
-                     kScaleRowBytes, &full_b[st]);
+            if constexpr (!kTrL2) {
+              bulk_g2s(dst + KG::kThumbOffset, src_p + static_cast<size_t>(tok) * kThumbRowBytes,
+                       kKvTok * kThumbRowBytes, &full_b[st]);
+              bulk_g2s(dst + KG::kScaleOffset, src_s + static_cast<size_t>(tok / T) * kHeadDim,
+                       kScaleRowBytes, &full_b[st]);
+            }
           } else {
             tma_load_3d(dst, &tmap_k, 0, y, 0, &full_b[st]);  // K: both halves
           }
@@ -720,6 +783,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int use = it_next / NKV;
           if (use > 0 && !mbar_test_wait(&empty_b[st], static_cast<uint32_t>(use - 1) & 1u)) break;
           meta[st] = -1;
+          if constexpr (kTrL2) __threadfence_block();
           seq[st] = it_next;
           mbar_arrive(&full_b[st]);
           ++it_next;
@@ -795,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // on it.  Decided here, after the pipeline has started, and published
     // (with the query group copied for the helpers) in ctrl[7].
     bool help = false;
-    if constexpr (C) {
+    if constexpr (kCoop) {
       // (both loads in flight together: the query group, 16 bytes x G x 16
       // over the lanes, and the split's previous bits)
       constexpr int kQv = (G * kHeadDim / 8 + 31) / 32;
@@ -1029,7 +1093,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // landed (the selector's work, decided in order by the scan warp).
     // (The scan warp publishes whether to help shortly after the start, so
     // the flag is read on every turn of the wait, one value for the warp.)
-    if (C && !dense) {
+    if (kCoop && !dense) {
       bool failed = false;
       uint64_t t0 = global_timer_ns();
       while (!__shfl_sync(kFull, lane == 0 ? seq[st] == it : 0, 0)) {
@@ -1061,66 +1125,78 @@ __global__ void __launch_bounds__(kThreads, 2)
     // a parity wait could then match that older phase.  The producer writes
     // `it` into seq[st] only after the previous fill was consumed, so once it
     // is visible the parity below names exactly this fill.
-    if (!wait_item_published(seq, st, it, p.wait_limit_ns) ||
-        !mbar_wait(&full_b[st], static_cast<uint32_t>(it / NKV) & 1u, p.wait_limit_ns)) {
+    if (!wait_item_published(seq, st, it, p.wait_limit_ns)) {
       raise_timeout(p, ctrl);
       break;
     }
-    const int tok = meta[st];
+    constexpr int MT = kKvTok / 16;
+    int tok = -1;
+    float sc0 = kScaleLog2, sc1 = kScaleLog2;  // logit scale of heads 2*t4, 2*t4 + 1
+    uint32_t qh[16];                           // thumbnail format: the folded query (f16 pairs)
+    uint2 thumb[MT][2];                        // thumbnail format: rows 16mt + gid (+8), words 2*t4 (+1)
+    if constexpr (kTrL2) {
+      __threadfence_block();  // pairs with the producer's fence between meta and seq
+      tok = meta[st];
+      // While the stage's residuals and values are in flight, load its
+      // thumbnail rows and its block's scale row from global memory (L2 after
+      // the scan) and fold the scales into the query.  (Plain coherent loads:
+      // the CTA that re-quantises the last block wrote these rows earlier in
+      // this launch.)
+      uint4 sv4[4] = {};
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) thumb[mt][0] = thumb[mt][1] = make_uint2(0u, 0u);
+      if (tok >= 0 &&
+          FFD_IN_BOUNDS(p, tok + kKvTok <= p.capacity && row < static_cast<size_t>(p.batch) * p.num_kv_heads)) {
+        const uint8_t *trow = p.packed + (row * p.capacity + static_cast<size_t>(tok)) * kThumbRowBytes + 8 * t4;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          thumb[mt][0] = *reinterpret_cast<const uint2 *>(trow + (16 * mt + gid) * kThumbRowBytes);
+          thumb[mt][1] = *reinterpret_cast<const uint2 *>(trow + (16 * mt + gid + 8) * kThumbRowBytes);
+        }
+        const uint4 *s4 =
+            reinterpret_cast<const uint4 *>(
+                p.scales + (row * static_cast<size_t>(p.capacity / T) + static_cast<size_t>(tok / T)) * kHeadDim) +
+            4 * t4;
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) sv4[w4] = s4[w4];
+      }
+      fold_query_tr(qb, t4, [&](int w4) { return sv4[w4]; }, qh, sc0, sc1);
+    }
+    if (!mbar_wait(&full_b[st], static_cast<uint32_t>(it / NKV) & 1u, p.wait_limit_ns)) {
+      raise_timeout(p, ctrl);
+      break;
+    }
+    if constexpr (!kTrL2) tok = meta[st];
     if (tok < 0) break;
     const uint32_t kbase = kv_ring_addr + st * KG::kStageBytes;
     const uint32_t vbase = kbase + KG::kVOffset;
 
     // S^T = K Q^T for kKvTok tokens: kKvTok/16 independent accumulator chains
-    constexpr int MT = kKvTok / 16;
     float sacc[MT][4];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) sacc[mt][0] = sacc[mt][1] = sacc[mt][2] = sacc[mt][3] = 0.0f;
-    float sc0 = kScaleLog2, sc1 = kScaleLog2;  // logit scale of heads 2*t4, 2*t4 + 1
     if constexpr (kTR) {
-      // Keys are rebuilt from thumbnail + residual as k_hat = s z / 254 with
-      // the integer z = 254 u - 381 + e (exact in f16).  The block's scales go
-      // into the query instead: q'_c = f16(q_c s_c 2^E / 254), E per head so
-      // that max |q'| is about 2^13 (no f16 overflow or underflow), and the
-      // scores are scaled back by 2^-E in fp32.
-      const uint8_t *stage = kv_ring + st * KG::kStageBytes;
-      const uint4 *s4 = reinterpret_cast<const uint4 *>(stage + KG::kScaleOffset) + 4 * t4;
-      float fq[32];
-      float am = 0.0f;
-#pragma unroll
-      for (int w4 = 0; w4 < 4; ++w4) {
-        const uint4 sv = s4[w4];
-        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * w4 + e;  // channel pair 32*t4 + 2i
-          const uint32_t qw = qb[i >> 1][i & 1];
-          fq[2 * i] = __fmul_rn(bf16_lo(qw), bf16_lo(sw[e]));
-          fq[2 * i + 1] = __fmul_rn(bf16_hi(qw), bf16_hi(sw[e]));
-          am = fmaxf(am, fmaxf(fabsf(fq[2 * i]), fabsf(fq[2 * i + 1])));
-        }
-      }
-      am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
-      am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
-      const int ea = static_cast<int>((__float_as_uint(am) >> 23) & 0xFFu);
-      const int E = min(148 - ea, 126);  // am 2^E in [2^21, 2^22)
-      const float mult = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 + E) << 23) * (1.0f / 254.0f);
-      const float uns = ea == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - E) << 23) * kScaleLog2;
-      uint32_t qh[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) qh[i] = pack_f16x2(fq[2 * i] * mult, fq[2 * i + 1] * mult);
-      sc0 = __shfl_sync(kFull, uns, (2 * t4) << 2);
-      sc1 = __shfl_sync(kFull, uns, (2 * t4 + 1) << 2);
       // Lane (gid, t4) supplies channels 32*t4 + 16h + {2k, 2k+1} (a0/a1) and
       // {2k+8, 2k+9} (a2/a3) at k-step (h, k): thumbnail word 2*t4 + h and
       // residual chunk 2*t4 + h of rows gid and gid + 8 (both rows = gid mod
       // 8, so the swizzle XOR is gid).
-      const uint8_t *thumb_s = stage + KG::kThumbOffset;
+      const uint8_t *stage = kv_ring + st * KG::kStageBytes;
+      if constexpr (!kTrL2) {  // the block's scales from the stage
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(stage + KG::kScaleOffset) + 4 * t4;
+        fold_query_tr(qb, t4, [&](int w4) { return s4[w4]; }, qh, sc0, sc1);
+      }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         const int r0 = 16 * mt + gid, r1 = r0 + 8;
-        const uint2 w0 = *reinterpret_cast<const uint2 *>(thumb_s + r0 * kThumbRowBytes + 8 * t4);
-        const uint2 w1 = *reinterpret_cast<const uint2 *>(thumb_s + r1 * kThumbRowBytes + 8 * t4);
+        uint2 w0, w1;  // thumbnail words 2*t4 (+1) of rows r0, r1
+        if constexpr (kTrL2) {
+          w0 = thumb[mt][0];
+          w1 = thumb[mt][1];
+        } else {
+          const uint8_t *thumb_s = stage + KG::kThumbOffset;
+          w0 = *reinterpret_cast<const uint2 *>(thumb_s + r0 * kThumbRowBytes + 8 * t4);
+          w1 = *reinterpret_cast<const uint2 *>(thumb_s + r1 * kThumbRowBytes + 8 * t4);
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int chunk = ((2 * t4 + h) ^ gid) << 4;
@@ -1383,8 +1459,9 @@ constexpr size_t smem_bytes_tf(int split_blocks) {
 constexpr size_t kSmemPerCta2 = (228 * 1024) / 2 - 1024;
 static_assert(smem_bytes_tf<64, kFormatInt4, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
 static_assert(smem_bytes_tf<128, kFormatInt4, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<64, kFormatThumbResid, false>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
 static_assert(smem_bytes_tf<64, kFormatThumbResid, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
-static_assert(smem_bytes_tf<128, kFormatThumbResid, true>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
+static_assert(smem_bytes_tf<128, kFormatThumbResid, false>(FFD_MAX_SPLIT_BLOCKS) <= kSmemPerCta2, "two CTAs per SM");
 
 // Raise the kernel's dynamic shared memory cap once per device, to the
 // largest split this library accepts, so later launches (and graph captures)
@@ -1405,17 +1482,16 @@ cudaError_t configure_tgfc() {
   return cudaSuccess;
 }
 
-// The variants of one (T, G, F): the int4 format has both selectors, the
-// thumbnail format only the scan warp's.
-// The cooperative selector is built for the int4 format's 64-token blocks
-// (at 128 tokens its registers spill); dense mode has no selector.
+// The variants of one (T, G, F): the sparse-step variant (C) is built for
+// 64-token blocks (at 128 tokens the cooperative selector's registers spill,
+// and a thumbnail split of 64 blocks is too long for its rows to stay in L2).
 template <int T, int F>
-constexpr bool kHasCoop = F == kFormatInt4 && T == 64;
+constexpr bool kHasSparseVariant = T == 64;
 
 template <int T, int G, int F>
 cudaError_t configure_tgf() {
   cudaError_t e = configure_tgfc<T, G, F, false>();
-  if (e == cudaSuccess && kHasCoop<T, F>) e = configure_tgfc<T, G, F, kHasCoop<T, F>>();
+  if (e == cudaSuccess && kHasSparseVariant<T, F>) e = configure_tgfc<T, G, F, kHasSparseVariant<T, F>>();
   return e;
 }
 
@@ -1429,12 +1505,15 @@ cudaError_t launch_tgfc(const DecodeParams &p, const CUtensorMap &tk, const CUte
   return cudaGetLastError();
 }
 
-// The cooperative selector is built for the int4 format's 64-token blocks
-// (at 128 tokens its registers spill); dense mode has no selector.
+// Dense steps have no selector and no scan (so nothing puts thumbnail rows in
+// L2 ahead of the computer); the thumbnail format's L2 loads pay only while a
+// split's scan runs a short way ahead of its computer (at most 4096 tokens).
 template <int T, int G, int F>
 cudaError_t launch_tgf(const DecodeParams &p, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
                        cudaStream_t stream) {
-  if (kHasCoop<T, F> && !p.dense) return launch_tgfc<T, G, F, kHasCoop<T, F>>(p, tk, tv, grid, stream);
+  const bool sparse_variant =
+      kHasSparseVariant<T, F> && !p.dense && (F == kFormatInt4 || p.split_blocks * T <= kTrL2MaxSplitTokens);
+  if (sparse_variant) return launch_tgfc<T, G, F, kHasSparseVariant<T, F>>(p, tk, tv, grid, stream);
   return launch_tgfc<T, G, F, false>(p, tk, tv, grid, stream);
 }
 
@@ -1482,9 +1561,10 @@ __global__ void bounds_selftest_kernel(DecodeParams p) {
 
 size_t decode_smem_bytes(int block_size, int group, int split_blocks, int format) {
   (void)group;
-  // the larger of a format's variants (the cooperative one for int4)
+  // the larger of a format's variants
   if (format == kFormatThumbResid)
-    return block_size == 64 ? smem_bytes_tf<64, kFormatThumbResid, false>(split_blocks)
+    return block_size == 64 ? std::max(smem_bytes_tf<64, kFormatThumbResid, false>(split_blocks),
+                                       smem_bytes_tf<64, kFormatThumbResid, true>(split_blocks))
                             : smem_bytes_tf<128, kFormatThumbResid, false>(split_blocks);
   return block_size == 64 ? smem_bytes_tf<64, kFormatInt4, true>(split_blocks)
                           : smem_bytes_tf<128, kFormatInt4, false>(split_blocks);

@@ -28,6 +28,9 @@ SMALL = [
     (6, 1, 4, 2, 8192, 64, 64, 5000, 8192),
     (7, 2, 4, 1, 4096, 64, 33, 1, 4096),
     (10, 2, 4, 2, 4480, 64, 64, 1, 4480),
+    # splits longer than 4096 tokens: the sparse steps keep the stage layout
+    # with thumbnail and scale rows inside the stage
+    (11, 1, 4, 2, 10240, 64, 80, 1, 10240),
 ]
 
 THUMB_POISON = 0x5A
