@@ -1103,39 +1103,46 @@ def run_context_sweep(args):
 
 
 def rho_row(name, ref_name, ref, device, steps, warmup, world, peak, l2, check=True, inp=None,
-            dense=False):
+            dense=False, fmt="int4"):
     """One row of the kept-fraction sweep: the fused step on a controlled-
-    sparsity workload (ffd_workloads.RHO_DOMINANT) with one reference maximum,
-    timed from CUDA graphs; optionally checked against the oracle (mask
-    bit-exact, output max-abs / mean-abs) on the same inputs."""
+    sparsity workload (ffd_workloads.RHO_DOMINANT) with one reference maximum
+    and key format, timed from CUDA graphs; optionally checked against the
+    oracle (mask bit-exact, output max-abs / mean-abs) on the same inputs."""
     import torch
     w = fw.WORKLOADS[name]
     if inp is None:
         inp = fw.make_inputs(w)
-    probe = Replica(w, inp, device, 1)
+    probe = Replica(w, inp, device, 1, fmt=fmt)
     probe.reference = ref
     probe.step(0, w.delta)
     torch.cuda.synchronize(device)
     mask = probe.layers[0]["bufs"].mask.cpu().numpy().view(np.uint32)
     out = probe.layers[0]["bufs"].out.float().cpu().numpy().astype(np.float64)
     kept_blocks, valid_blocks, kept_tok = kept_tokens_from_mask(w, inp["lengths"], mask)
-    algo = algorithmic_bytes(w, inp["lengths"], kept_tok, dense=False)["total"]
+    algo = (algorithmic_bytes_tr if fmt == "tr" else algorithmic_bytes)(w, inp["lengths"], kept_tok,
+                                                                        dense=False)["total"]
     del probe
-    row = {"workload": name, "reference": ref_name,
+    row = {"workload": name, "format": fmt, "reference": ref_name,
            "kept_fraction": kept_blocks / max(1, valid_blocks), "algorithmic_bytes": algo}
     if check:
         import oracle
-        packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
-        sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
-        _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
-                                     w.split_blocks, w.delta, reference=ref)
-        want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
-                                    w.block_size)
+        if fmt == "tr":
+            thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], w.block_size)
+            want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales,
+                                                      inp["lengths"], w.block_size, w.split_blocks,
+                                                      w.delta, reference=ref)
+        else:
+            packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+            sc = oracle.block_scores(inp["q"], packed, scales, inp["lengths"], w.block_size)
+            _, want_mask = oracle.select(sc, inp["lengths"], w.num_kv_heads, w.capacity, w.block_size,
+                                         w.split_blocks, w.delta, reference=ref)
+            want_out, _ = oracle.attend(inp["q"], inp["k"], inp["v"], inp["lengths"], want_mask,
+                                        w.block_size)
         err = np.abs(out - want_out)
         row["oracle"] = {"mask_equal": bool(np.array_equal(mask, want_mask)),
                          "max_abs": float(err.max()), "mean_abs": float(err.mean())}
     layers = max(1, min(64, math.ceil(3 * l2 / algo)))
-    rep = Replica(w, inp, device, layers)
+    rep = Replica(w, inp, device, layers, fmt=fmt)
     rep.reference = ref
     _, per, _ = time_graph_steps(rep, w.delta, steps, warmup, world, device)
     us = dist_max(float(np.mean(per)) * 1e3, world, device)
@@ -1164,19 +1171,23 @@ def run_rho_sweep(args):
     peak, peak_src = load_peaks()
     refs = [("running", REFERENCES["running"]), ("sink_local_fixed", REFERENCES["sink_local_fixed"])]
     rows = []
-    dense_us = None
+    dense_us = {}
     steps = min(args.steps, 400)
+    # int4 with both references, then the thumbnail format (the pages' own key
+    # split) with the running maximum
+    legs = [("int4", ref_name, ref) for ref_name, ref in refs] + [("tr", "running", REFERENCES["running"])]
     for name in fw.RHO_DOMINANT:
         inp = fw.make_inputs(fw.WORKLOADS[name])
-        for ref_name, ref in refs:
+        for fmt, ref_name, ref in legs:
             row = rho_row(name, ref_name, ref, device, steps, args.warmup, 1, peak, l2, check=True,
-                          inp=inp, dense=dense_us is None)
-            dense_us = row.get("dense_us", dense_us)
-            row["dense_us"] = dense_us
-            row["vs_dense"] = dense_us / row["decode_us"]
+                          inp=inp, dense=fmt not in dense_us, fmt=fmt)
+            dense_us[fmt] = row.get("dense_us", dense_us.get(fmt))
+            row["dense_us"] = dense_us[fmt]
+            row["vs_dense"] = dense_us[fmt] / row["decode_us"]
             rows.append(row)
         del inp
-    line = {"mode": "rho-sweep", "metric": "us per decode launch vs kept fraction (128K)",
+    line = {"mode": "rho-sweep", "metric": "us per decode launch vs kept fraction (128K), int4 and "
+                                          "thumbnail + residual key formats",
             "unit": "us",
             "workload": "long-context shape (B1 Hq32 Hkv8 D128 N131072 T64 S64 delta 3) with "
                         "concentrated attention: keys 0.1 N(0,1), n of every 64 blocks raised by "

@@ -111,15 +111,15 @@ struct KvGeom<kFormatThumbResid, true> {
   static constexpr int kStages = 7;
 };
 
-// With the cooperative selector (int4, C) the ring has as many stages as fit
-// beside the K/V ring with two CTAs per SM, since several warps hold stages at
-// once; with the scan warp alone, fewer.
+// With the cooperative selector (C) the ring has as many stages as fit beside
+// the K/V ring with two CTAs per SM, since several warps hold stages at once;
+// with the scan warp alone, fewer.
 template <int T, int F, bool C>
 struct ScanGeom {
   static constexpr int kRowBytes = F == kFormatThumbResid ? kThumbRowBytes : kPackedRowBytes;
   static constexpr int kStageBytes = T * kRowBytes + kScaleRowBytes;
-  static constexpr int kStages = F == kFormatThumbResid ? 2 * (T == 64 ? 4 : 2)
-                                                        : (C ? (T == 64 ? 6 : 3) : (T == 64 ? 4 : 2));
+  static constexpr int kStages = C ? (F == kFormatThumbResid ? (T == 64 ? 9 : 5) : (T == 64 ? 6 : 3))
+                                   : (F == kFormatThumbResid ? 2 : 1) * (T == 64 ? 4 : 2);
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kRingBytes >= kMergeBytes, "merge scratch aliases the scan ring");
 };
@@ -575,12 +575,12 @@ __device__ __forceinline__ void fold_query_tr(const uint32_t (&qb)[8][2], int t4
   sc1 = __shfl_sync(kFull, uns, (2 * t4 + 1) << 2);
 }
 
-// C: the sparse-step variant for 64-token blocks.  int4 format: the
-// cooperative selector (the attention warps score scan entries while they wait
-// for K/V); without it (dense mode) the scan warp scores every entry itself.
-// Thumbnail format (splits of at most 4096 tokens): the attention stages leave
-// out the thumbnail rows and scale rows, which the attention warps load from
-// L2 (KvGeom); its selector is always the scan warp's.
+// C: the sparse-step variant for 64-token blocks: the cooperative selector
+// (the attention warps score scan entries while they wait for K/V); without it
+// (dense mode, 128-token blocks) the scan warp scores every entry itself.  In
+// the thumbnail format (splits of at most 4096 tokens) the variant's attention
+// stages also leave out the thumbnail rows and scale rows, which the attention
+// warps load from L2 (KvGeom).
 template <int T, int G, int F, bool C>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   using SL = SmemLayout<T, F, C>;
   using KG = KvGeom<F, C>;
   constexpr bool kTR = F == kFormatThumbResid;
-  constexpr bool kCoop = C && !kTR;  // the cooperative selector
+  constexpr bool kCoop = C;          // the cooperative selector
   constexpr bool kTrL2 = C && kTR;   // thumbnails and scales from L2
   constexpr int NSA = SG::kStages;
   constexpr int NKV = KG::kStages;
@@ -853,11 +853,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     // Cooperative selector: the attention warps help the scan unless this
     // CTA's share of the split's kept blocks in the previous call on this
     // workspace (the split's selection bits are still there, and a part
-    // attends over 1 / R of them) was at least 3/4 of the split: then the
+    // attends over 1 / R of them) was at least 3/4 of the split (int4) or 1/8
+    // (thumbnails, whose attention warps also rebuild every key): then the
     // attention warps are the bound and the scan warp keeps ahead alone.
     // This only spreads the work; the selection and the output do not depend
-    // on it.  Decided here, after the pipeline has started, and published
-    // (with the query group copied for the helpers) in ctrl[7].
+    // on it.  Decided here, after the pipeline has started, and published in
+    // ctrl[7]: 1 = help (the query group is copied for the helpers first),
+    // 2 = no help (the attention warps then wait plainly).
     bool help = false;
     if constexpr (kCoop) {
       // (both loads in flight together: the query group, 16 bytes x G x 16
@@ -874,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         prev += __popc(__ldcg(p.split_bits + (row * p.nsplit_max + split) * p.split_words + w));
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) prev += __shfl_xor_sync(kFull, prev, off);
-      help = 4 * prev < 3 * nbs * R;  // (a part attends over 1 / R of the kept blocks)
+      help = kTR ? 8 * prev < nbs * R : 4 * prev < 3 * nbs * R;  // (a part attends over 1 / R of them)
       if (help) {
 #pragma unroll
         for (int k = 0; k < kQv; ++k)
@@ -884,6 +886,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           __threadfence_block();
           ctrl[7] = 1;
         }
+      } else if (lane == 0) {
+        ctrl[7] = 2;
       }
     }
     if (!help) {
@@ -1087,18 +1091,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int v_chi = (lane >> 3) & 1;
   const uint32_t kv_ring_addr = smem_addr(kv_ring);
 
+  bool coop_wait = kCoop && !dense;  // until the scan warp says that this CTA does not help
   for (int it = warp;; it += kAttnWarps) {
     const int st = it % NKV;
     // Until item `it` is published, score scan entries whose tiles have
     // landed (the selector's work, decided in order by the scan warp).
     // (The scan warp publishes whether to help shortly after the start, so
     // the flag is read on every turn of the wait, one value for the warp.)
-    if (kCoop && !dense) {
+    if (coop_wait) {
       bool failed = false;
       uint64_t t0 = global_timer_ns();
       while (!__shfl_sync(kFull, lane == 0 ? seq[st] == it : 0, 0)) {
-        const bool help = __shfl_sync(kFull, lane == 0 ? ctrl[7] : 0, 0) != 0;
-        const int e = help ? claim_scan_entry<NSA>(sh, full_a, nref + nbs, true, lane) : -2;
+        const int flag = __shfl_sync(kFull, lane == 0 ? ctrl[7] : 0, 0);
+        if (flag == 2) {  // no help in this call: wait plainly from now on
+          coop_wait = false;
+          break;
+        }
+        const int e = flag == 1 ? claim_scan_entry<NSA>(sh, full_a, nref + nbs, true, lane) : -2;
         if (e == -1) break;  // every entry is taken: wait for the item alone
         if (e >= 0) {
           const int jb = scan_block_index(e, nref, nb, j0);
