@@ -306,3 +306,34 @@ def test_decode_tr_short_context_shares_splits_between_ctas(delta):
     assert_mask_equal(mask, want_mask, f"tr 16K {delta}")
     assert_output_close(out, want_out, f"tr 16K {delta}")
     assert ffd.check_device_status(tc.bufs.workspace) == 0
+
+
+@pytest.mark.parametrize("batch", [4, 1])
+def test_decode_tr_kept_fraction_and_call_history_do_not_change_results(batch):
+    # The controlled-sparsity workloads at a 32K context on one workspace,
+    # calls alternating between 1/64 and all blocks kept: the sparse variant's
+    # per-call helper switch (from the previous call's selection bits; the
+    # thumbnail format helps below 1/8 kept) runs both ways, with one CTA per
+    # split (B4) and two (B1).  Every call must match the oracle.
+    cases = []
+    for name in ("rho1of64", "rho1"):
+        w = fw.scaled_workload(fw.WORKLOADS[name], batch=batch, capacity=32768, context=32768)
+        inp = fw.make_inputs(w)
+        thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], w.block_size)
+        want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales,
+                                                  inp["lengths"], w.block_size, w.split_blocks, w.delta)
+        cases.append((name, w, inp, want_out, want_mask))
+    ws = None
+    for name, w, inp, want_out, want_mask in cases + cases + cases[:1]:
+        tc = TrCase(w, inp)
+        if ws is None:
+            ws = tc.bufs.workspace
+        tc.quantize(0)
+        ffd.decode_tr(tc.shape, tc.q, tc.k, tc.v, tc.bufs.k_thumb, tc.bufs.k_resid, tc.bufs.k_scales,
+                      tc.lengths, w.delta, tc.bufs.out, tc.bufs.mask, ws, requant_last=True)
+        torch.cuda.synchronize()
+        out = bf16_to_np_f32(tc.bufs.out).astype(np.float64)
+        mask = tc.bufs.mask.cpu().numpy().view(np.uint32)
+        assert_mask_equal(mask, want_mask, f"tr {name} B{batch}")
+        assert_output_close(out, want_out, f"tr {name} B{batch}")
+        assert ffd.check_device_status(ws) == 0
