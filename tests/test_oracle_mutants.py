@@ -27,6 +27,8 @@ MUTANTS = [
     ("topdelta-no-group-union", "if (k) m[j / 32] |= 1u << (j % 32);",
      "if (k && h % G == 0) m[j / 32] |= 1u << (j % 32);", 0),
     ("pseudo-fixed-sink-only", "float pseudo = fmaxf(s[0], s[nb - 1]);", "float pseudo = s[0];", 1),
+    ("pseudo-seeded-no-running-update", "running = fmaxf(running, s[j]);", "(void)running;", 1),
+    ("query-fold-range", "float inv = 127.0f / a;", "float inv = 128.0f / a;", 0),
     ("attention-no-scale", "double scale = 1.0 / sqrt((double)D);", "double scale = 1.0;", 0),
     ("attention-denominator", "o[c] /= denom;", "o[c] /= denom + 1.0;", 0),
     ("attention-gqa-map",
@@ -34,6 +36,7 @@ MUTANTS = [
      "      int g = h % Hkv;\n      size_t row = (size_t)b * Hkv + g;\n      const uint16_t *qh", 0),
     ("thumb-level-step", "(double)(254 * u - 381 + e) / 254.0", "(double)(256 * u - 381 + e) / 254.0", 0),
     ("thumb-score-offset", "(2 * thumb_code(tr, c) - 3)", "(2 * thumb_code(tr, c) - 2)", 0),
+    ("thumb-residual-step", "nearbyintf(d * 254.0f)", "nearbyintf(d * 256.0f)", 0),
 ]
 
 
