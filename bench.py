@@ -952,13 +952,15 @@ def run_gpu(args):
 
     # the method's own regime beside the headline: the same shape with
     # concentrated attention, where few blocks are kept (timing only; the
-    # oracle checks these rows in --rho-sweep and in the GPU tests)
+    # oracle checks these rows in --rho-sweep and in the GPU tests), int4 and
+    # the thumbnail format
     rho = None
     if not args.no_rho:
         rho = [rho_row(name, ref_name, REFERENCES[ref_name], device, min(args.steps, 200),
-                       min(args.warmup, 10), world, load_peaks()[0], l2, check=False)
-               for name, ref_name in (("rho1of64", "running"), ("rho0p05", "running"),
-                                      ("rho1of64", "sink_local_fixed"))]
+                       min(args.warmup, 10), world, load_peaks()[0], l2, check=False, fmt=fmt)
+               for name, ref_name, fmt in (("rho1of64", "running", "int4"), ("rho0p05", "running", "int4"),
+                                           ("rho1of64", "sink_local_fixed", "int4"),
+                                           ("rho1of64", "running", "tr"))]
 
     e2e = None
     if not args.no_e2e:
