@@ -428,3 +428,24 @@ def test_short_context_shares_splits_between_ctas(context, delta):
         assert_mask_equal(gc.bufs.mask.cpu().numpy().view(np.uint32), want_mask, f"{context} {delta}")
         assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, f"{context} {delta}")
     assert ffd.check_device_status(gc.bufs.workspace) == 0
+
+
+@pytest.mark.parametrize("name", ["rho1of64", "rho0p25"])
+def test_controlled_sparsity_at_full_size(name):
+    # The 128K long-context shape with n of every 64 blocks raised above the
+    # rest (the kept-fraction sweep's inputs, same seeds), in the launch the
+    # sweep times: the fused step against the oracle, mask bit-exact.
+    from gpu_util import bf16_to_np_f32
+    w = fw.WORKLOADS[name]
+    inp = fw.make_inputs(w)
+    packed, scales = oracle.quantize_keys(inp["k"], inp["lengths"], w.block_size)
+    want_out, want_mask, _ = oracle.decode(inp["q"], inp["k"], inp["v"], packed, scales, inp["lengths"],
+                                           w.block_size, w.split_blocks, w.delta)
+    gc = GpuCase(w, inp)
+    gc.quantize(0)
+    ffd.decode_ex(gc.shape, gc.q, gc.k, gc.v, gc.bufs.k_packed, gc.bufs.k_scales, gc.lengths, w.delta,
+                  gc.bufs.out, gc.bufs.mask, gc.bufs.workspace, requant_last=True)
+    torch.cuda.synchronize()
+    assert_mask_equal(gc.bufs.mask.cpu().numpy().view(np.uint32), want_mask, name)
+    assert_output_close(bf16_to_np_f32(gc.bufs.out).astype(np.float64), want_out, name)
+    assert ffd.check_device_status(gc.bufs.workspace) == 0

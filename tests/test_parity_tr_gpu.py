@@ -337,3 +337,20 @@ def test_decode_tr_kept_fraction_and_call_history_do_not_change_results(batch):
         assert_mask_equal(mask, want_mask, f"tr {name} B{batch}")
         assert_output_close(out, want_out, f"tr {name} B{batch}")
         assert ffd.check_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("name", ["rho1of64", "rho0p25"])
+def test_decode_tr_controlled_sparsity_at_full_size(name):
+    # The kept-fraction sweep's thumbnail rows at full size (128K, same
+    # seeds): the fused step against the oracle, mask bit-exact.
+    w = fw.WORKLOADS[name]
+    inp = fw.make_inputs(w)
+    thumb, resid, scales = oracle.quantize_keys_tr(inp["k"], inp["lengths"], w.block_size)
+    want_out, want_mask, _ = oracle.decode_tr(inp["q"], inp["v"], thumb, resid, scales, inp["lengths"],
+                                              w.block_size, w.split_blocks, w.delta)
+    tc = TrCase(w, inp)
+    tc.quantize(0)
+    out, mask = tc.decode(w.delta, requant_last=True)
+    assert_mask_equal(mask, want_mask, f"tr {name}")
+    assert_output_close(out, want_out, f"tr {name}")
+    assert ffd.check_device_status(tc.bufs.workspace) == 0
