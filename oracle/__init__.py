@@ -1,7 +1,7 @@
 """ctypes wrapper of the plain C oracle (``ffd_oracle.c``).
 
 TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
-CPU-baseline leg are the only callers.  The product path never imports this
+CPU-baseline leg and CPU reference arm are the only callers.  The product path never imports this
 package, and this package imports nothing from the product.
 
 All arrays are numpy: bf16 tensors are passed as their uint16 bit patterns.

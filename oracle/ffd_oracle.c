@@ -3,8 +3,8 @@
  * decode path.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check of the graft
- * entry module and the benchmark's CPU-baseline leg may load or call this
- * library.  The product path (the CUDA library and its Python binding) never
+ * entry module and the benchmark's CPU-baseline leg and CPU reference arm may
+ * load or call this library.  The product path (the CUDA library and its Python binding) never
  * does, and this file shares no code, header, table or constant with it.
  *
  * Source of the method: "Faster Than Flash: Exploiting Attention Sparsity for
